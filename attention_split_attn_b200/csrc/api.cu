@@ -1,0 +1,365 @@
+// api.cu -- the C ABI of libattn_b200 (declared in include/attn.h):
+// argument validation, the slice planner, workspace sizing, TMA descriptors,
+// the device status word, and dispatch to the kernel launchers.
+//
+// Refusal instead of a wrong result: every shape, dtype, stride or workspace
+// the kernels do not cover is rejected here before any launch (the
+// supports_op refusal of strix-llama.cpp PR #115: a backend declines an op it
+// cannot compute rather than computing it wrongly; TensorFold PR #2595's
+// launch guard: a grid is launched only where it stays inside the buffers).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "attn.h"
+#include "internal.h"
+
+namespace attn {
+namespace {
+
+thread_local std::string g_last_error;
+
+int32_t fail(int32_t status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+int dtype_size(int32_t t) {
+  switch (t) {
+    case ATTN_F32: return 4;
+    case ATTN_F16: return 2;
+    case ATTN_BF16: return 2;
+    default: return 0;
+  }
+}
+
+// ---- device facts ------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  int* status = nullptr;   // device address of g_status_word on this device
+};
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+}  // namespace
+}  // namespace attn
+
+// One status word per device, written by kernels that gave up on a bounded wait.
+__device__ int g_status_word = 0;
+
+namespace attn {
+namespace {
+
+int32_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(ATTN_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return fail(ATTN_ERR_CUDA, "cannot query device %d", dev);
+    if (major != 10 || minor != 0)
+      return fail(ATTN_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                  major, minor);
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess)
+      return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    d.status = static_cast<int*>(addr);
+    d.init = true;
+  }
+  *out = &d;
+  return ATTN_OK;
+}
+
+// ---- TMA descriptors ---------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+CUtensorMapDataType tma_dtype(int32_t t) {
+  switch (t) {
+    case ATTN_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    case ATTN_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    default: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  }
+}
+
+// 3-D map over a [cells][heads][D] cache: box = (D, 1, box_cells).
+int32_t make_kv_map(CUtensorMap* map, const void* base, int32_t type, int D, int Hkv, int N,
+                    int64_t stride_cell, int64_t stride_head, int box_cells) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int es = dtype_size(type);
+  // A stride of an extent-1 dimension is never used; give the encoder a legal one.
+  const int64_t sh = Hkv > 1 ? stride_head : D;
+  const int64_t sc = N > 1 ? stride_cell : D;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)N};
+  cuuint64_t strides[2] = {(cuuint64_t)(sh * es), (cuuint64_t)(sc * es)};
+  cuuint32_t box[3] = {(cuuint32_t)D, 1u, (cuuint32_t)box_cells};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, tma_dtype(type), 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ATTN_OK;
+}
+
+// ---- validation ----------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t validate_common(const attn_args* a, int32_t op) {
+  if (!a) return fail(ATTN_ERR_INVALID_ARG, "args is NULL");
+  for (int i = 0; i < 5; ++i)
+    if (a->reserved[i] != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved fields must be zero");
+  if (a->n_rows < 0 || a->n_cells < 0) return fail(ATTN_ERR_INVALID_ARG, "negative n_rows or n_cells");
+  if (a->n_head_q <= 0 || a->n_head_kv <= 0)
+    return fail(ATTN_ERR_INVALID_ARG, "n_head_q and n_head_kv must be positive");
+  if (a->n_head_q % a->n_head_kv != 0)
+    return fail(ATTN_ERR_INVALID_ARG, "n_head_q (%d) is not a multiple of n_head_kv (%d)", a->n_head_q,
+                a->n_head_kv);
+  if (!dtype_size(a->q_type) || !dtype_size(a->kv_type) || !dtype_size(a->out_type))
+    return fail(ATTN_ERR_INVALID_ARG, "unknown dtype");
+  if (a->head_dim != 64 && a->head_dim != 128 && a->head_dim != 256)
+    return fail(ATTN_ERR_UNSUPPORTED, "head_dim %d not in {64, 128, 256}", a->head_dim);
+  const int G = a->n_head_q / a->n_head_kv;
+  if (G > 16) return fail(ATTN_ERR_UNSUPPORTED, "GQA group %d > 16", G);
+  if ((a->row_begin == nullptr) != (a->row_end == nullptr))
+    return fail(ATTN_ERR_INVALID_ARG, "row_begin and row_end must both be given or both be NULL");
+  if ((a->cell_seq == nullptr) != (a->row_seq == nullptr))
+    return fail(ATTN_ERR_INVALID_ARG, "cell_seq and row_seq must both be given or both be NULL");
+  if (a->causal != 0 && a->causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (a->mask && a->mask_stride_row < 0) return fail(ATTN_ERR_INVALID_ARG, "negative mask stride");
+  if (a->n_slices < 0 || a->n_slices > 64) return fail(ATTN_ERR_INVALID_ARG, "n_slices must be 0..64");
+  if (a->max_row_len < 0) return fail(ATTN_ERR_INVALID_ARG, "negative max_row_len");
+  if (a->grid_order != 0 && a->grid_order != 1) return fail(ATTN_ERR_INVALID_ARG, "grid_order must be 0 or 1");
+  if (!(a->scale == a->scale)) return fail(ATTN_ERR_INVALID_ARG, "scale is NaN");
+  if (a->n_rows == 0) return ATTN_OK;
+  if (!a->q || !a->out) return fail(ATTN_ERR_INVALID_ARG, "q or out is NULL");
+  if (a->n_cells > 0 && (!a->k || !a->v)) return fail(ATTN_ERR_INVALID_ARG, "k or v is NULL");
+  if (a->q_stride_row < 0 || a->q_stride_head < 0 || a->o_stride_row < 0 || a->o_stride_head < 0 ||
+      a->kv_stride_cell < 0 || a->kv_stride_head < 0)
+    return fail(ATTN_ERR_INVALID_ARG, "negative stride");
+  const int es = dtype_size(a->kv_type);
+  if (a->n_cells > 0) {
+    if (!aligned16(a->k) || !aligned16(a->v))
+      return fail(ATTN_ERR_UNSUPPORTED, "k and v must be 16-byte aligned");
+    if ((a->kv_stride_cell * es) % 16 || (a->kv_stride_head * es) % 16)
+      return fail(ATTN_ERR_UNSUPPORTED, "kv strides must be multiples of 16 bytes");
+    if ((a->n_cells > 1 && a->kv_stride_cell == 0) || (a->n_head_kv > 1 && a->kv_stride_head == 0))
+      return fail(ATTN_ERR_UNSUPPORTED, "zero kv stride (broadcast caches are not supported)");
+  }
+  (void)op;
+  return ATTN_OK;
+}
+
+// ---- decode planning -------------------------------------------------------------
+constexpr int kSliceGrain = 32;     // slices are cut at multiples of 32 cells
+
+struct DecodeShape {
+  int32_t S, C, hpw, hg;
+};
+
+int pick_hpw(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
+
+DecodeShape plan_decode(const attn_args* a, int sms) {
+  DecodeShape d;
+  const int G = a->n_head_q / a->n_head_kv;
+  d.hg = G > 8 ? 2 : 1;
+  d.hpw = G > 8 ? 8 : pick_hpw(G);
+  int64_t max_len = a->max_row_len > 0 ? std::min(a->max_row_len, a->n_cells) : a->n_cells;
+  max_len = std::max<int64_t>(max_len, 1);
+  int64_t S = a->n_slices;
+  if (S == 0) {
+    // Slices of about 256 cells (128 KB of bf16 K+V at D 128 per CTA), but no
+    // more CTAs than ~16 per SM in total, and at most 64 slices.
+    const int64_t units = (int64_t)a->n_rows * a->n_head_kv;
+    S = (max_len + 255) / 256;
+    const int64_t cap = std::max<int64_t>(1, (16LL * std::max(sms, 1)) / std::max<int64_t>(units, 1));
+    S = std::min(S, cap);
+    S = std::min<int64_t>(std::max<int64_t>(S, 1), 64);
+  }
+  int64_t C = (max_len + S - 1) / S;
+  C = (C + kSliceGrain - 1) / kSliceGrain * kSliceGrain;
+  d.S = (int32_t)S;
+  d.C = (int32_t)std::max<int64_t>(C, kSliceGrain);
+  return d;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t decode_ws_bytes(const attn_args* a, const DecodeShape& d) {
+  if (d.S <= 1) return 0;
+  const size_t slots = (size_t)a->n_rows * a->n_head_q * d.S;
+  return align256(slots * a->head_dim * sizeof(float)) + align256(slots * 2 * sizeof(float));
+}
+
+int32_t check_decode(const attn_args* a) {
+  int32_t st = validate_common(a, ATTN_OP_DECODE);
+  if (st != ATTN_OK) return st;
+  const int G = a->n_head_q / a->n_head_kv;
+  if (!decode_shape_supported(a->kv_type, a->head_dim, G))
+    return fail(ATTN_ERR_UNSUPPORTED, "decode: unsupported kv dtype/head_dim/group");
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int32_t attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+const char* attn_strerror(int32_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT";
+    default: return "unknown attn_status";
+  }
+}
+
+const char* attn_last_error(void) { return g_last_error.c_str(); }
+
+int32_t attn_supports(const attn_args* a, int32_t op) {
+  switch (op) {
+    case ATTN_OP_DECODE: return check_decode(a);
+    default: return fail(ATTN_ERR_UNSUPPORTED, "op %d is not available in this build", op);
+  }
+}
+
+size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
+  (void)n_sel;
+  if (attn_supports(a, op) != ATTN_OK) return 0;
+  int sms = 148;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) == ATTN_OK) sms = di->sms;
+  switch (op) {
+    case ATTN_OP_DECODE: return decode_ws_bytes(a, plan_decode(a, sms));
+    default: return 0;
+  }
+}
+
+int32_t attn_decode(const attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  int32_t st = check_decode(a);
+  if (st != ATTN_OK) return st;
+  if (a->n_rows == 0) return ATTN_OK;
+  DeviceInfo* di = nullptr;
+  if ((st = device_info(&di)) != ATTN_OK) return st;
+  const DecodeShape sh = plan_decode(a, di->sms);
+  const size_t need = decode_ws_bytes(a, sh);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(ATTN_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
+  if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(ATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const int64_t blocks = (int64_t)a->n_rows * a->n_head_kv * sh.S;
+  if (blocks > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid of %lld CTAs is too large", (long long)blocks);
+
+  CUtensorMap tmK, tmV;
+  memset(&tmK, 0, sizeof(tmK));
+  memset(&tmV, 0, sizeof(tmV));
+  if (a->n_cells > 0) {
+  if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                        a->kv_stride_head, 32)) != ATTN_OK)
+    return st;
+  if ((st = make_kv_map(&tmV, a->v, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                        a->kv_stride_head, 32)) != ATTN_OK)
+    return st;
+  }
+
+  DecodePlan p{};
+  p.R = a->n_rows; p.Hq = a->n_head_q; p.Hkv = a->n_head_kv; p.G = a->n_head_q / a->n_head_kv;
+  p.D = a->head_dim; p.N = a->n_cells;
+  p.q = QSpec{a->q, a->q_type, a->q_stride_row, a->q_stride_head};
+  p.out = OutSpec{a->out, a->out_type, a->o_stride_row, a->o_stride_head};
+  p.f = RowFilter{a->row_begin, a->row_end, a->cell_seq, a->row_seq, a->cell_pos, a->row_pos,
+                  a->causal, a->mask, a->mask_stride_row};
+  p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
+  p.S = sh.S; p.C = sh.C; p.grid_order = a->grid_order;
+  p.hpw = sh.hpw; p.hg = sh.hg; p.kv_type = a->kv_type;
+  p.status = di->status;
+  if (sh.S > 1) {
+    const size_t slots = (size_t)a->n_rows * a->n_head_q * sh.S;
+    p.part.o = static_cast<float*>(ws);
+    p.part.ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(slots * a->head_dim * sizeof(float)));
+    p.part.S = sh.S;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode(p, tmK, tmV, s);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  if (sh.S > 1) {
+    ReducePlan rp{};
+    rp.R = a->n_rows; rp.Hq = a->n_head_q; rp.D = a->head_dim;
+    rp.out = p.out; rp.sinks = a->sinks; rp.part = p.part;
+    rp.row_begin = a->row_begin; rp.row_end = a->row_end; rp.N = a->n_cells; rp.C = sh.C;
+    rp.n_used = nullptr; rp.use_pdl = 1;
+    e = launch_split_k_reduce(rp, s);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "split_k_reduce launch: %s", cudaGetErrorString(e));
+  }
+  return ATTN_OK;
+}
+
+int32_t attn_selected(const attn_selected_args* a, void* ws, size_t ws_bytes, void* stream) {
+  (void)a; (void)ws; (void)ws_bytes; (void)stream;
+  return fail(ATTN_ERR_UNSUPPORTED, "attn_selected is not available in this build");
+}
+
+int32_t attn_prefill(const attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  (void)a; (void)ws; (void)ws_bytes; (void)stream;
+  return fail(ATTN_ERR_UNSUPPORTED, "attn_prefill is not available in this build");
+}
+
+int32_t attn_check_device_status(void* stream) {
+  DeviceInfo* di = nullptr;
+  int32_t st = device_info(&di);
+  if (st != ATTN_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA, "stream synchronize failed");
+  int word = 0;
+  if (cudaMemcpy(&word, di->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA, "cannot read the device status word");
+  if (word != 0) {
+    const int zero = 0;
+    cudaMemcpy(di->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(word, "a kernel reported %s", attn_strerror(word));
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"

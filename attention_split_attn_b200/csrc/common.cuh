@@ -1,0 +1,218 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of libattn_b200.
+//
+// mbarrier waits are bounded: a wait that does not complete within
+// kWaitLimitNs records ATTN_ERR_DEVICE_TIMEOUT in the caller's status word and
+// returns false, so a kernel never spins forever.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "attn.h"
+
+namespace attn {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// arithmetic
+// ---------------------------------------------------------------------------
+
+// max that returns NaN if either input is NaN (fmaxf drops NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// 2^x on the special-function unit: 2^-inf = +0, 2^NaN = NaN.
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+__device__ __forceinline__ float qnan() { return __int_as_float(0x7fffffff); }
+
+// ---------------------------------------------------------------------------
+// storage types
+// ---------------------------------------------------------------------------
+
+template <typename T> struct Storage;
+template <> struct Storage<float> { static constexpr int kDtype = ATTN_F32; };
+template <> struct Storage<__half> { static constexpr int kDtype = ATTN_F16; };
+template <> struct Storage<__nv_bfloat16> { static constexpr int kDtype = ATTN_BF16; };
+
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+__device__ __forceinline__ void unpack_f16x2(uint32_t w, float& lo, float& hi) {
+  __half2 h = *reinterpret_cast<__half2*>(&w);
+  float2 f = __half22float2(h);
+  lo = f.x; hi = f.y;
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const uint4& w, float* f) {
+  if constexpr (sizeof(T) == 4) {
+    f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+    f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+  } else if constexpr (Storage<T>::kDtype == ATTN_BF16) {
+    unpack_bf16x2(w.x, f[0], f[1]); unpack_bf16x2(w.y, f[2], f[3]);
+    unpack_bf16x2(w.z, f[4], f[5]); unpack_bf16x2(w.w, f[6], f[7]);
+  } else {
+    unpack_f16x2(w.x, f[0], f[1]); unpack_f16x2(w.y, f[2], f[3]);
+    unpack_f16x2(w.z, f[4], f[5]); unpack_f16x2(w.w, f[6], f[7]);
+  }
+}
+
+// One element of a runtime-typed array, widened exactly to float.
+__device__ __forceinline__ float load_as_float(const void* base, int64_t i, int dtype) {
+  if (dtype == ATTN_F32) return static_cast<const float*>(base)[i];
+  if (dtype == ATTN_F16) return __half2float(static_cast<const __half*>(base)[i]);
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
+}
+
+// Round-to-nearest-even store of a float into a runtime-typed array.
+__device__ __forceinline__ void store_from_float(void* base, int64_t i, int dtype, float x) {
+  if (dtype == ATTN_F32) static_cast<float*>(base)[i] = x;
+  else if (dtype == ATTN_F16) static_cast<__half*>(base)[i] = __float2half_rn(x);
+  else static_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------------------
+// status word
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// shared memory, mbarrier, TMA
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete, for at most about
+// kWaitLimitNs.  Returns false (and records a timeout) if it never does.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      record_status(status, ATTN_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// 3-D tiled TMA load into shared memory, completing on `bar` (tx bytes).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(c0), "r"(c1), "r"(c2), "l"(cache_hint)
+      : "memory");
+}
+
+// Contiguous bulk copy global -> shared (16-byte aligned, size multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// L2 eviction-priority policies for cache_hint operands.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Named barrier over a subset of warps (id 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue / wait for the previous kernel's results.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// host: opt a kernel into more than 48 KB of dynamic shared memory, once per
+// device (the attribute is per function and per device context).
+// ---------------------------------------------------------------------------
+// `done` must be a static owned by the caller's kernel instantiation (one
+// bit per device).
+template <typename Kernel>
+inline cudaError_t set_smem_limit_once(std::atomic<unsigned long long>& done, Kernel kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+}  // namespace attn

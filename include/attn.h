@@ -1,0 +1,171 @@
+/*
+ * attn.h -- C ABI of libattn_b200: attention over a KV cache on B200 (sm_100a).
+ *
+ * Three operations share one argument block and one set of semantics:
+ *
+ *   attn_decode    split-K decode.  Work is cut into (row, KV head, slice)
+ *                  units on a (rows, heads, slices) grid; each unit runs an
+ *                  online softmax over its slice for every query head of the
+ *                  KV head (GQA sharing), and a split_k_reduce pass folds the
+ *                  slice partials.  Defined by TensorFold PR #2595 ("attn_decode
+ *                  grid becomes (rows, heads, slices)"; attn_decode + attn_merge
+ *                  registered as one operator: Q rows, K/V cache -> attention
+ *                  rows; 32-key slices).
+ *   attn_selected  maskless selected-key attention: a query row sees exactly
+ *                  the cells named in its selection list; the list is sorted,
+ *                  invalid and duplicate entries are skipped, and K/V are
+ *                  gathered in blocks of 32 cells; rows are split into parts
+ *                  combined by split_k_reduce when the grid would under-fill
+ *                  the GPU.  Defined by strix-llama.cpp PR #115 / #119
+ *                  (FLASH_ATTN_EXT with a selection list src[5];
+ *                  flash_attn_sel.comp; flash_attn_split_k_reduce).
+ *   attn_prefill   causal prefill: many query rows over the cache, QK^T and PV
+ *                  on the tensor cores, same semantics as decode.
+ *
+ * Semantics (all three; HartsyInference PR #910 "attention semantic
+ * correctness"):  for row r and query head h (KV head g = h / (Hq/Hkv)),
+ *   x_c = scale * q.k_c;  x_c = softcap*tanh(x_c/softcap) if softcap > 0;
+ *   then x_c += slope_h * -|row_pos - cell_pos| (ALiBi, after the softcap);
+ *   then x_c += mask[r,c] in F32, never narrowed;
+ *   sigma = sinks[h] (an extra logit with no value vector) or -inf;
+ *   out = sum_c exp(x_c - M) v_c / (sum_c exp(x_c - M) + exp(sigma - M)),
+ *   M = max(x, sigma); a row with no visible cell (and sigma = -inf or
+ *   finite) is +0.0; NaN anywhere among the logits or the sink gives NaN in
+ *   every element; NaN in a visible V gives NaN in that element, also across
+ *   the split combine; +inf logit or sink gives NaN.
+ *
+ * Visibility of cell c for row r (decode and prefill):
+ *   row_begin[r] <= c < row_end[r]            (NULL: [0, n_cells))
+ *   and cell_seq[c] == row_seq[r]             (if both are non-NULL)
+ *   and cell_pos[c] <= row_pos[r]             (if causal)
+ *   and mask[r, c] != -inf                    (if mask; a -inf cell is never read)
+ * Positions: cell_pos NULL -> c - row_begin[r]; row_pos NULL ->
+ * row_end[r] - row_begin[r] - 1.  Selected: the distinct entries e of row r's
+ * list with 0 <= e < n_cells; no range, sequence, causal or mask filter.
+ *
+ * Memory and ownership.  Every pointer in the argument blocks is DEVICE
+ * memory owned by the caller.  The caller also owns the workspace (sized by
+ * attn_workspace_size) and the stream.  The library allocates nothing per
+ * call, never synchronizes in attn_decode/attn_selected/attn_prefill, and is
+ * asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ * default stream).  Arguments are read during the call; the argument block
+ * may be reused as soon as the call returns.
+ *
+ * Errors.  Every call returns an attn_status.  A shape, dtype, stride or
+ * workspace the kernels do not cover is refused with ATTN_ERR_UNSUPPORTED or
+ * ATTN_ERR_INVALID_ARG before anything is launched (never a wrong result);
+ * attn_last_error() gives a one-line reason (thread-local).  The library
+ * never aborts or traps.  Kernels that wait on a barrier give up after a
+ * bounded number of polls and record ATTN_ERR_DEVICE_TIMEOUT in a device
+ * status word, read by attn_check_device_status().
+ *
+ * Layouts (strides in ELEMENTS; the head dimension is contiguous):
+ *   q   [n_rows][n_head_q][head_dim]      q_stride_row, q_stride_head
+ *   k,v [n_cells][n_head_kv][head_dim]    kv_stride_cell, kv_stride_head (shared by k and v)
+ *   out [n_rows][n_head_q][head_dim]      o_stride_row, o_stride_head
+ *   mask [n_rows][n_cells] F32            mask_stride_row
+ * K and V base addresses and their cell/head strides must be 16-byte
+ * aligned (tile loads by the Tensor Memory Accelerator).
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_ABI_VERSION 1
+
+typedef enum { ATTN_F32 = 0, ATTN_F16 = 1, ATTN_BF16 = 2 } attn_dtype;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = -1,     /* null/negative/inconsistent argument           */
+    ATTN_ERR_UNSUPPORTED = -2,     /* valid, but not a shape/dtype the kernels take  */
+    ATTN_ERR_WORKSPACE = -3,       /* workspace missing or smaller than required     */
+    ATTN_ERR_CUDA = -4,            /* a CUDA runtime call failed (launch, attribute) */
+    ATTN_ERR_DEVICE_TIMEOUT = -5   /* a kernel gave up waiting on a barrier          */
+} attn_status;
+
+enum { ATTN_OP_DECODE = 0, ATTN_OP_SELECTED = 1, ATTN_OP_PREFILL = 2 };
+
+/* Shared argument block (see the file comment for meaning and layout). */
+typedef struct {
+    int32_t n_rows, n_head_q, n_head_kv, head_dim, n_cells;
+
+    const void *q;   int32_t q_type;   int64_t q_stride_row, q_stride_head;
+    const void *k;   const void *v;    int32_t kv_type;
+    int64_t kv_stride_cell, kv_stride_head;
+    void *out;       int32_t out_type; int64_t o_stride_row, o_stride_head;
+
+    const int32_t *row_begin, *row_end;   /* [n_rows] or NULL                       */
+    const int32_t *cell_seq, *row_seq;    /* [n_cells], [n_rows] or NULL            */
+    const int32_t *cell_pos, *row_pos;    /* [n_cells], [n_rows] or NULL            */
+    int32_t causal;                       /* 0/1                                     */
+    const float *mask; int64_t mask_stride_row;   /* F32 [n_rows][n_cells] or NULL  */
+
+    float scale;                          /* applied to q.k before everything else  */
+    float softcap;                        /* <= 0: off                               */
+    const float *alibi_slopes;            /* [n_head_q] or NULL                      */
+    const float *sinks;                   /* [n_head_q] or NULL (= -inf)             */
+
+    int32_t n_slices;     /* decode: 0 = from occupancy; else 1..64 slices per row  */
+    int32_t max_row_len;  /* decode: host-side upper bound on row_end - row_begin
+                             (sizes the slices); 0 = unknown, n_cells is used.  A
+                             longer row is still correct: its last slice takes the
+                             excess.                                                 */
+    int32_t grid_order;   /* 0: rows vary fastest over the (rows, heads, slices)
+                             grid; 1: slices fastest.  Results are bit-identical;
+                             exposed for tests and tuning.                           */
+    int32_t reserved[5];  /* must be zero                                            */
+} attn_args;
+
+/* Selected-key arguments.  base.row_begin/row_end/cell_seq/row_seq/mask must be
+ * NULL and base.causal 0 (the op is maskless; visibility is the list alone).
+ * cell_pos/row_pos are still used for ALiBi distances.                       */
+typedef struct {
+    attn_args base;
+    const int32_t *sel;       /* [n_rows][sel_stride_row], first n_sel used      */
+    int64_t sel_stride_row;
+    int32_t n_sel;            /* 1..4096 entries per row                          */
+    int32_t *sel_sorted_out;  /* optional [n_rows][n_sel]: valid distinct entries
+                                 ascending, then -1 padding                        */
+    int32_t *sel_count_out;   /* optional [n_rows]: number of distinct valid entries */
+} attn_selected_args;
+
+/* Workspace bytes the op needs for these arguments (0 is possible).  n_sel is
+ * used by ATTN_OP_SELECTED only.  Returns 0 also for invalid arguments; call
+ * attn_supports() to tell the two apart.                                     */
+size_t attn_workspace_size(const attn_args *args, int32_t op, int32_t n_sel);
+
+/* ATTN_OK if the op takes these arguments, else the status the op would
+ * return (nothing is launched).                                              */
+int32_t attn_supports(const attn_args *args, int32_t op);
+
+/* The three operations.  ws/ws_bytes: device workspace of at least
+ * attn_workspace_size() bytes, 256-byte aligned (may be NULL when 0 bytes are
+ * needed).  Contents on entry are irrelevant; on return they are scratch.
+ * Two calls that share a workspace must be ordered on the GPU.             */
+int32_t attn_decode(const attn_args *args, void *ws, size_t ws_bytes, void *stream);
+int32_t attn_selected(const attn_selected_args *args, void *ws, size_t ws_bytes, void *stream);
+int32_t attn_prefill(const attn_args *args, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronizes `stream`, then reads and clears the device status word on the
+ * current device: ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on
+ * a bounded wait since the last check.                                      */
+int32_t attn_check_device_status(void *stream);
+
+/* Human-readable name of a status; reason of the last refusal on this thread. */
+const char *attn_strerror(int32_t status);
+const char *attn_last_error(void);
+
+/* ATTN_ABI_VERSION of the loaded library. */
+int32_t attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ATTN_B200_H */

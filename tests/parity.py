@@ -1,0 +1,77 @@
+"""Comparison of the CUDA path with the FP64 oracle.
+
+Acceptance (element by element, on the same seeded inputs):
+  * the NaN positions of the output and the oracle are identical;
+  * where the oracle is exactly 0 (a fully excluded row) the output is +0.0;
+  * over the finite oracle values, NMSE = sum (out-ref)^2 / sum ref^2 is at
+    most 1e-10 when Q, K, V and the output are all FP32, and at most 1e-5
+    with max |out - ref| <= 2e-2 otherwise (FP16/BF16 storage or output).
+The 1e-10 bound is for logits of moderate size: an FP32 logit carries an
+absolute error of about ulp(|x|), so an FP32 kernel cannot do better than
+exp(ulp(|x|)) relative on a weight whatever its design.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import attention_split_attn_b200 as A
+
+
+def tolerance(p):
+    all_f32 = (p.q.dtype == torch.float32 and p.k.dtype == torch.float32
+               and p.out_dtype == torch.float32)
+    return (1e-10, None) if all_f32 else (1e-5, 2e-2)
+
+
+def compare(got, ref, nmse_tol, max_abs=None, what=""):
+    got = got.detach().to(torch.float64).cpu().numpy() if isinstance(got, torch.Tensor) else got
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    gn, rn = np.isnan(got), np.isnan(ref)
+    if not np.array_equal(gn, rn):
+        idx = np.argwhere(gn != rn)[:5]
+        raise AssertionError(f"{what}: NaN pattern differs at {idx.tolist()} "
+                             f"(got {[got[tuple(i)] for i in idx]}, ref {[ref[tuple(i)] for i in idx]})")
+    zero = (ref == 0.0)
+    if zero.any():
+        gz = got[zero]
+        assert np.all(gz == 0.0) and not np.signbit(gz).any(), \
+            f"{what}: excluded elements not +0.0: {gz[(gz != 0) | np.signbit(gz)][:5]}"
+    fin = np.isfinite(ref)
+    assert np.all(np.isfinite(got[fin])), f"{what}: non-finite output where the oracle is finite"
+    num = float(np.sum((got[fin] - ref[fin]) ** 2))
+    den = float(np.sum(ref[fin] ** 2))
+    nmse = num / den if den > 0 else num
+    assert nmse <= nmse_tol, f"{what}: NMSE {nmse:.3e} > {nmse_tol:.1e}"
+    if max_abs is not None and fin.any():
+        err = float(np.max(np.abs(got[fin] - ref[fin])))
+        assert err <= max_abs, f"{what}: max abs error {err:.3e} > {max_abs}"
+    return nmse
+
+
+def check(p, got, what="", ref=None):
+    ref = oracle.attn(p) if ref is None else ref
+    tol, max_abs = tolerance(p)
+    return compare(got, ref, tol, max_abs, what)
+
+
+def poisoned_workspace(nbytes, device="cuda"):
+    """A workspace whose every float is NaN, so any slot a kernel reads
+    without having written it shows up in the output."""
+    if nbytes == 0:
+        return None
+    return torch.full((nbytes,), 0xFF, dtype=torch.uint8, device=device)
+
+
+def run_decode(p, **over):
+    (q, k, v, out), kw = A.problem_kwargs(p)
+    kw.update(over)
+    out.fill_(float("nan"))
+    args = A.make_args(q, k, v, out, **kw)
+    ws = poisoned_workspace(A.workspace_size(args, A.OP_DECODE))
+    A.attn_decode_args(args, ws=ws)
+    torch.cuda.synchronize()
+    A.check_device_status()
+    return out
