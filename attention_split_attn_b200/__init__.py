@@ -31,8 +31,8 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
-           "attn_prefill", "attn_check_device_status", "attn_strerror", "attn_last_error",
-           "attn_abi_version")
+           "attn_prefill", "attn_decode_timed", "attn_check_device_status", "attn_strerror",
+           "attn_last_error", "attn_abi_version")
 
 
 class AttnArgs(ctypes.Structure):
@@ -94,6 +94,9 @@ def load_library():
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int32
                 fn.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            lib.attn_decode_timed.restype = ctypes.c_int32
+            lib.attn_decode_timed.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t,
+                                              ctypes.c_void_p, ctypes.c_void_p * 3]
             lib.attn_selected.restype = ctypes.c_int32
             lib.attn_selected.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
                                           ctypes.c_size_t, ctypes.c_void_p]
@@ -196,6 +199,20 @@ def attn_decode_args(args: AttnArgs, ws: Optional[torch.Tensor] = None, stream=N
                          0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
     _raise_if(st, "attn_decode")
     return ws
+
+
+def attn_decode_timed_args(args: AttnArgs, ws: Optional[torch.Tensor], events, stream=None):
+    """attn_decode that also records three torch.cuda.Events (before the slice
+    kernel, after it, after split_k_reduce) on the launching stream."""
+    lib = load_library()
+    handles = [None if e is None else e.cuda_event for e in events]
+    if any(h == 0 for h in handles):
+        raise ValueError("record each torch.cuda.Event once before passing it (torch creates it lazily)")
+    ev = (ctypes.c_void_p * 3)(*handles)
+    st = lib.attn_decode_timed(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                               0 if ws is None else ws.numel() * ws.element_size(),
+                               _stream_handle(stream), ev)
+    _raise_if(st, "attn_decode_timed")
 
 
 def decode(q, k, v, out, *, ws=None, stream=None, **kw):

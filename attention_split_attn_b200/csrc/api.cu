@@ -116,9 +116,11 @@ CUtensorMapDataType tma_dtype(int32_t t) {
   }
 }
 
-// 3-D map over a [cells][heads][D] cache: box = (D, 1, box_cells).
+// 3-D map over a [cells][heads][D] cache: box = (box_d, 1, box_cells); with
+// swizzle the box rows are 128 bytes and stored with the 128-byte swizzle.
 int32_t make_kv_map(CUtensorMap* map, const void* base, int32_t type, int D, int Hkv, int N,
-                    int64_t stride_cell, int64_t stride_head, int box_cells) {
+                    int64_t stride_cell, int64_t stride_head, int box_cells, int box_d = 0,
+                    bool swizzle128 = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int es = dtype_size(type);
@@ -127,10 +129,11 @@ int32_t make_kv_map(CUtensorMap* map, const void* base, int32_t type, int D, int
   const int64_t sc = N > 1 ? stride_cell : D;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)N};
   cuuint64_t strides[2] = {(cuuint64_t)(sh * es), (cuuint64_t)(sc * es)};
-  cuuint32_t box[3] = {(cuuint32_t)D, 1u, (cuuint32_t)box_cells};
+  cuuint32_t box[3] = {(cuuint32_t)(box_d > 0 ? box_d : D), 1u, (cuuint32_t)box_cells};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(map, tma_dtype(type), 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return ATTN_OK;
@@ -188,22 +191,32 @@ int32_t validate_common(const attn_args* a, int32_t op) {
 constexpr int kSliceGrain = 32;     // slices are cut at multiples of 32 cells
 
 struct DecodeShape {
+  bool mma;       // tensor-core kernels (16-bit cache, Q in the cache dtype)
+  bool stream;    // balanced persistent scheme (mma and no forced slice count)
   int32_t S, C, hpw, hg;
+  int32_t W;      // balanced scheme: warps of the persistent grid
 };
 
 int pick_hpw(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
 
+// Two schemes.  With the tensor-core kernels and no forced slice count, every
+// resident warp takes an equal run of the flattened (row, KV head, 16-cell
+// tile) space (decode_stream.cu).  Otherwise the (rows, heads, slices) grid:
+// S slices per row (forced, or about 256 cells each, at most 16 CTAs per SM
+// in all and at most 64 slices), each C cells long on the 32-cell grid, the
+// last slice taking whatever remains of a longer row.
 DecodeShape plan_decode(const attn_args* a, int sms) {
   DecodeShape d;
   const int G = a->n_head_q / a->n_head_kv;
+  d.mma = decode_uses_mma(a->kv_type, a->q_type, a->q, a->q_stride_row, a->q_stride_head);
+  d.stream = d.mma && a->n_slices == 0;
   d.hg = G > 8 ? 2 : 1;
   d.hpw = G > 8 ? 8 : pick_hpw(G);
+  d.W = d.stream ? decode_stream_warps(a->kv_type, a->head_dim, G, sms) : 0;
   int64_t max_len = a->max_row_len > 0 ? std::min(a->max_row_len, a->n_cells) : a->n_cells;
   max_len = std::max<int64_t>(max_len, 1);
   int64_t S = a->n_slices;
   if (S == 0) {
-    // Slices of about 256 cells (128 KB of bf16 K+V at D 128 per CTA), but no
-    // more CTAs than ~16 per SM in total, and at most 64 slices.
     const int64_t units = (int64_t)a->n_rows * a->n_head_kv;
     S = (max_len + 255) / 256;
     const int64_t cap = std::max<int64_t>(1, (16LL * std::max(sms, 1)) / std::max<int64_t>(units, 1));
@@ -212,18 +225,36 @@ DecodeShape plan_decode(const attn_args* a, int sms) {
   }
   int64_t C = (max_len + S - 1) / S;
   C = (C + kSliceGrain - 1) / kSliceGrain * kSliceGrain;
-  d.S = (int32_t)S;
+  d.S = d.stream ? 0 : (int32_t)S;
   d.C = (int32_t)std::max<int64_t>(C, kSliceGrain);
   return d;
 }
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-size_t decode_ws_bytes(const attn_args* a, const DecodeShape& d) {
-  if (d.S <= 1) return 0;
-  const size_t slots = (size_t)a->n_rows * a->n_head_q * d.S;
-  return align256(slots * a->head_dim * sizeof(float)) + align256(slots * 2 * sizeof(float));
+// Workspace layout: [row_tiles (balanced scheme)] [partial o records] [partial (m, l)].
+struct DecodeWs {
+  size_t tiles_off, o_off, ml_off, total;
+};
+
+DecodeWs decode_ws_layout(const attn_args* a, const DecodeShape& d) {
+  DecodeWs w{0, 0, 0, 0};
+  const int G = a->n_head_q / a->n_head_kv;
+  size_t records;
+  if (d.stream) {
+    w.tiles_off = 0;
+    w.o_off = align256(((size_t)a->n_rows + 1) * sizeof(int64_t));
+    records = ((size_t)d.W + (size_t)a->n_rows * a->n_head_kv) * G;
+  } else {
+    if (d.S <= 1) return w;
+    records = (size_t)a->n_rows * a->n_head_q * d.S;
+  }
+  w.ml_off = w.o_off + align256(records * a->head_dim * sizeof(float));
+  w.total = w.ml_off + align256(records * 2 * sizeof(float));
+  return w;
 }
+
+size_t decode_ws_bytes(const attn_args* a, const DecodeShape& d) { return decode_ws_layout(a, d).total; }
 
 int32_t check_decode(const attn_args* a) {
   int32_t st = validate_common(a, ATTN_OP_DECODE);
@@ -276,7 +307,20 @@ size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
   }
 }
 
+namespace attn {
+namespace {
+void record_event(void* const* events, int i, cudaStream_t s) {
+  if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+}
+}  // namespace
+}  // namespace attn
+
 int32_t attn_decode(const attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  return attn_decode_timed(a, ws, ws_bytes, stream, nullptr);
+}
+
+int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* stream,
+                          void* const events[3]) {
   int32_t st = check_decode(a);
   if (st != ATTN_OK) return st;
   if (a->n_rows == 0) return ATTN_OK;
@@ -288,19 +332,21 @@ int32_t attn_decode(const attn_args* a, void* ws, size_t ws_bytes, void* stream)
     return fail(ATTN_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
   if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(ATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  const int64_t blocks = (int64_t)a->n_rows * a->n_head_kv * sh.S;
+  const int64_t blocks = sh.stream ? sh.W : (int64_t)a->n_rows * a->n_head_kv * sh.S;
   if (blocks > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid of %lld CTAs is too large", (long long)blocks);
 
+  const bool mma = sh.mma;
   CUtensorMap tmK, tmV;
   memset(&tmK, 0, sizeof(tmK));
   memset(&tmV, 0, sizeof(tmV));
   if (a->n_cells > 0) {
-  if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
-                        a->kv_stride_head, 32)) != ATTN_OK)
-    return st;
-  if ((st = make_kv_map(&tmV, a->v, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
-                        a->kv_stride_head, 32)) != ATTN_OK)
-    return st;
+    const int box_d = mma ? 64 : 0;
+    if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                          a->kv_stride_head, mma ? 16 : 32, box_d, mma)) != ATTN_OK)
+      return st;
+    if ((st = make_kv_map(&tmV, a->v, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                          a->kv_stride_head, mma ? 16 : 32, box_d, mma)) != ATTN_OK)
+      return st;
   }
 
   DecodePlan p{};
@@ -312,26 +358,44 @@ int32_t attn_decode(const attn_args* a, void* ws, size_t ws_bytes, void* stream)
                   a->causal, a->mask, a->mask_stride_row};
   p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
   p.S = sh.S; p.C = sh.C; p.grid_order = a->grid_order;
-  p.hpw = sh.hpw; p.hg = sh.hg; p.kv_type = a->kv_type;
+  p.hpw = sh.hpw; p.hg = sh.hg; p.kv_type = a->kv_type; p.mma = mma ? 1 : 0;
   p.status = di->status;
-  if (sh.S > 1) {
-    const size_t slots = (size_t)a->n_rows * a->n_head_q * sh.S;
-    p.part.o = static_cast<float*>(ws);
-    p.part.ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(slots * a->head_dim * sizeof(float)));
+  const DecodeWs wl = decode_ws_layout(a, sh);
+  char* wsb = static_cast<char*>(ws);
+  if (wl.total > 0) {
+    p.part.o = reinterpret_cast<float*>(wsb + wl.o_off);
+    p.part.ml = reinterpret_cast<float*>(wsb + wl.ml_off);
     p.part.S = sh.S;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_decode(p, tmK, tmV, s);
-  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-  if (sh.S > 1) {
-    ReducePlan rp{};
-    rp.R = a->n_rows; rp.Hq = a->n_head_q; rp.D = a->head_dim;
-    rp.out = p.out; rp.sinks = a->sinks; rp.part = p.part;
-    rp.row_begin = a->row_begin; rp.row_end = a->row_end; rp.N = a->n_cells; rp.C = sh.C;
-    rp.n_used = nullptr; rp.use_pdl = 1;
-    e = launch_split_k_reduce(rp, s);
-    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "split_k_reduce launch: %s", cudaGetErrorString(e));
+  if (sh.stream) {
+    p.W = sh.W;
+    p.row_tiles = reinterpret_cast<int64_t*>(wsb + wl.tiles_off);
   }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  record_event(events, 0, s);
+  cudaError_t e;
+  if (sh.stream) {
+    e = launch_decode_stream(p, tmK, tmV, s, events ? static_cast<cudaEvent_t>(events[1]) : nullptr);
+  } else {
+    e = launch_decode_slices(p, tmK, tmV, s);
+    record_event(events, 1, s);
+  }
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  if (sh.stream || sh.S > 1) {
+    CombinePlan cp{};
+    cp.R = a->n_rows; cp.Hq = a->n_head_q; cp.Hkv = a->n_head_kv; cp.G = p.G; cp.D = a->head_dim;
+    cp.out = p.out; cp.sinks = a->sinks; cp.part = p.part;
+    cp.mode = sh.stream ? 1 : 0;
+    cp.row_begin = a->row_begin; cp.row_end = a->row_end; cp.N = a->n_cells; cp.C = sh.C;
+    cp.n_used = nullptr;
+    cp.row_tiles = p.row_tiles; cp.W = p.W;
+    // PDL overlap is off when the caller asked for an event between the two
+    // kernels: the event must see the main kernel complete.
+    cp.use_pdl = (events && events[1]) ? 0 : 1;
+    e = launch_combine(cp, s);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  }
+  record_event(events, 2, s);
   return ATTN_OK;
 }
 

@@ -1,5 +1,5 @@
-// decode.cu -- split-K decode attention (attn_decode) and the split_k_reduce
-// combine, for sm_100a.
+// decode_slice.cu -- split-K decode attention on a (rows, heads, slices) grid
+// (attn_decode with a forced slice count, and every FP32 or mixed-dtype cache).
 //
 // Work decomposition (TensorFold PR #2595, "What this changes": the
 // attn_decode grid is (rows, heads, slices) so that rows sharing a key slice
@@ -7,32 +7,35 @@
 // not depend on the grid order, so outputs are bit-identical across orders).
 // One CTA = one (row r, KV head g, slice s).  The slice is a run of cells of
 // row r cut at multiples of 32 cells from row_begin[r] (32-key slices, same
-// page, int8 crossover discussion); the CTA computes, for every query head of
-// KV head g (GQA sharing), the online-softmax partial (m, l, o[D]) of its
-// slice, and split_k_reduce folds the partials of a row in slice order with
-// the sink (attn_merge on the same page; flash_attn_split_k_reduce in
-// strix-llama.cpp PR #119).  With one slice per row the CTA folds the sink
-// itself and writes the row.
+// page); the CTA computes, for every query head of KV head g (GQA sharing),
+// the online-softmax partial (m, l, o[D]) of its slice, and the combine
+// (combine.cu) folds the partials of a row in slice order with the sink
+// (attn_merge on the same page; flash_attn_split_k_reduce in strix-llama.cpp
+// PR #119).  With one slice per row the CTA folds the sink itself and writes
+// the row.
 //
-// Data path (B200): one producer warp streams 32-cell K and V tiles of the
-// slice into a 4-stage shared-memory ring with 3-D TMA tile loads completing
-// on mbarriers (L2 evict-first: the cache is read once).  Four consumer warps
-// (per group of up to 8 query heads) score keys from shared memory with
-// 16-byte vector reads: LPK lanes cover one key's head_dim row, the dot
-// product is reduced with warp shuffles, and each (warp, lane group) keeps
-// its own running (m, l, o) over the keys it owns -- one max per 32-cell tile
-// (the tile-wise max of TensorFold PR #985, "64-key softmax tiles").  The
-// streams are merged in a fixed order at the end, so the result depends only
-// on the slice, never on scheduling.
+// Two kernels:
+//  * decode_slice_kernel (any cache dtype, CUDA cores): one producer warp
+//    streams 32-cell K and V tiles into a 4-stage ring with 3-D TMA loads on
+//    mbarriers; four consumer warps (per group of up to 8 q heads) score keys
+//    from shared memory with 16-byte vector reads, LPK lanes per key row and a
+//    shuffle reduction of the dot product; each (warp, lane group) keeps its
+//    own running (m, l, o) with one max per 32-cell tile (TensorFold PR #985,
+//    "64-key softmax tiles"); the streams are merged in a fixed order.
+//  * decode_warp_kernel (16-bit cache, Q in the cache dtype): a CTA is one
+//    warp that streams 16-cell tiles of its slice through a 3-stage TMA ring
+//    and folds them with tensor-core MMAs (decode_tile.cuh).
 //
 // Semantics (HartsyInference PR #910): the max propagates NaN; exp(-inf - -inf)
 // is guarded (an all -inf stream uses 0 as its reference); excluded cells
 // (outside the slice, other sequence, causal, mask == -inf) never contribute,
-// not even through 0 * NaN, because their V vector is zeroed before the FMA;
-// visible cells always contribute p * v, so a NaN in a visible V reaches the
-// output even when p underflows to 0.
+// not even through 0 * NaN, because their V vector is zeroed; visible cells
+// always contribute p * v, so a NaN in a visible V reaches the output even
+// when p underflows to 0.
 #include "common.cuh"
+#include "decode_tile.cuh"
 #include "internal.h"
+#include "mma.cuh"
 
 namespace attn {
 
@@ -71,37 +74,6 @@ struct DecodeSmem {
   static constexpr int kBarOffset = (kDataBytes + 127) / 128 * 128;
   static constexpr int kTotal = kBarOffset + 2 * Geo::NSTAGE * 8 + 16;
 };
-
-struct RowCtx {
-  int32_t begin, end;        // the row's cell range
-  int32_t s_begin, s_end;    // this slice
-  int32_t row_seq;
-  int64_t row_pos;
-};
-
-__device__ __forceinline__ bool cell_visible(const RowFilter& f, const RowCtx& rc, int r, int c,
-                                             float& mval, int64_t& cpos) {
-  bool vis = true;
-  if (f.cell_seq != nullptr && f.row_seq != nullptr) vis = (__ldg(f.cell_seq + c) == rc.row_seq);
-  cpos = f.cell_pos ? (int64_t)__ldg(f.cell_pos + c) : (int64_t)(c - rc.begin);
-  if (f.causal) vis = vis && (cpos <= rc.row_pos);
-  mval = 0.f;
-  if (f.mask != nullptr) {
-    mval = __ldg(f.mask + (int64_t)r * f.mask_sr + c);
-    vis = vis && !(mval == neg_inf());
-  }
-  return vis;
-}
-
-// Final fold of one (row, head): slice state (M, L, O) with the sink.
-__device__ __forceinline__ float fold_with_sink(float M, float L, float O, float sigma) {
-  const float Mf = fmax_nan(M, sigma);
-  if (isnan(Mf)) return qnan();
-  if (Mf == neg_inf()) return 0.f;
-  const float f = ex2((M - Mf) * kLog2e);
-  const float Lf = L * f + ex2((sigma - Mf) * kLog2e);
-  return (O * f) / Lf;
-}
 
 template <typename KT, int D, int HPW, int HG>
 __global__ void __launch_bounds__(32 * (kKeyWarps * HG + 1))
@@ -368,7 +340,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       store_from_float(p.out.out, (int64_t)r * p.out.sr + (int64_t)hq * p.out.sh + d, p.out.type,
                        fold_with_sink(M, L, O, sigma));
     } else {
-      const int64_t slot = ((int64_t)r * p.Hq + hq) * p.S + s;
+      const int64_t slot = (((int64_t)r * p.Hkv + g) * p.S + s) * G + hh;
       p.part.o[slot * D + d] = O;
       if (d == 0) {
         p.part.ml[slot * 2] = M;
@@ -378,58 +350,109 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   }
 }
 
-// ---- split_k_reduce --------------------------------------------------------
-// One warp per (row, q head); lanes stride over head_dim.  Slices are read in
-// order; NaN in any slice's m, or in the sink, gives NaN; a row whose max is
-// -inf is +0; otherwise out = sum_s o_s e^(m_s-M) / (sum_s l_s e^(m_s-M) + e^(sigma-M)).
-__global__ void __launch_bounds__(256) split_k_reduce_kernel(const ReducePlan p) {
-  pdl_wait_prior_grid();
-  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= (int64_t)p.R * p.Hq) return;
-  const int r = (int)(wid / p.Hq), h = (int)(wid % p.Hq);
-  int n_used;
-  if (p.n_used) {
-    n_used = min(__ldg(p.n_used + r), p.part.S);
+template <int D>
+struct WarpRing {
+  static constexpr int NS = (D <= 128) ? 3 : 2;      // ring stages
+  static constexpr int BAR_OFF = NS * WarpStage<D>::BYTES;
+  static constexpr int TOTAL = BAR_OFF + NS * 8 + 1024;   // + alignment slack for the swizzle
+};
+
+template <typename KT, int D, int NH>
+__global__ void __launch_bounds__(32)
+decode_warp_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const DecodePlan p) {
+  constexpr int NS = WarpRing<D>::NS;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + WarpRing<D>::BAR_OFF);
+  const int lane = threadIdx.x;
+
+  const int64_t bid = blockIdx.x;
+  int r, g, s;
+  if (p.grid_order == 0) {
+    r = (int)(bid % p.R);
+    g = (int)((bid / p.R) % p.Hkv);
+    s = (int)(bid / ((int64_t)p.R * p.Hkv));
   } else {
-    int32_t b = p.row_begin ? __ldg(p.row_begin + r) : 0;
-    int32_t e = p.row_end ? __ldg(p.row_end + r) : p.N;
-    b = max(b, 0);
-    e = min(e, p.N);
-    const int64_t len = e > b ? (int64_t)e - b : 0;
-    n_used = len == 0 ? 0 : (int)min((int64_t)p.part.S, (len + p.C - 1) / p.C);
+    s = (int)(bid % p.S);
+    g = (int)((bid / p.S) % p.Hkv);
+    r = (int)(bid / ((int64_t)p.S * p.Hkv));
   }
-  const int64_t base = ((int64_t)r * p.Hq + h) * p.part.S;
-  const float sigma = p.sinks ? __ldg(p.sinks + h) : neg_inf();
-  float M = sigma;
-  for (int s = 0; s < n_used; ++s) M = fmax_nan(M, p.part.ml[(base + s) * 2]);
-  const int64_t obase = (int64_t)r * p.out.sr + (int64_t)h * p.out.sh;
-  if (isnan(M) || M == neg_inf()) {
-    const float val = isnan(M) ? qnan() : 0.f;
-    for (int d = lane; d < p.D; d += 32) store_from_float(p.out.out, obase + d, p.out.type, val);
+  RowCtx rc;
+  rc.begin = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
+  rc.end = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
+  rc.begin = max(rc.begin, 0);
+  rc.end = min(rc.end, p.N);
+  if (rc.end < rc.begin) rc.end = rc.begin;
+  {
+    const int64_t b = rc.begin, e = rc.end;
+    const int64_t sb = b + (int64_t)s * p.C;
+    const int64_t se = (s == p.S - 1) ? e : min(e, sb + p.C);
+    rc.s_begin = (int32_t)min(sb, e);
+    rc.s_end = (int32_t)max(min(se, e), (int64_t)rc.s_begin);
+  }
+  if (p.S > 1 && rc.s_begin >= rc.s_end) {
+    pdl_launch_dependents();
     return;
   }
-  float L = ex2((sigma - M) * kLog2e);
-  constexpr int kMaxPerLane = 8;   // head_dim <= 256
-  float O[kMaxPerLane];
-#pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) O[i] = 0.f;
-  for (int s = 0; s < n_used; ++s) {
-    const float ms = p.part.ml[(base + s) * 2];
-    const float f = ex2((ms - M) * kLog2e);
-    L = fmaf(p.part.ml[(base + s) * 2 + 1], f, L);
-    const float* os = p.part.o + (base + s) * p.D;
-#pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-      const int d = lane + 32 * i;
-      if (d < p.D) O[i] = fmaf(os[d], f, O[i]);
+  rc.row_seq = p.f.row_seq ? __ldg(p.f.row_seq + r) : 0;
+  rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + r) : (int64_t)(rc.end - rc.begin - 1);
+  const bool has_filter = (p.f.cell_seq && p.f.row_seq) || p.f.causal || p.f.mask;
+  const int n_tiles = (rc.s_end - rc.s_begin + kWarpTile - 1) / kWarpTile;
+
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  pdl_launch_dependents();
+  uint64_t pol = 0;
+  if (lane == 0) {
+    pol = policy_evict_first();
+    for (int t = 0; t < min(NS, n_tiles); ++t)
+      issue_warp_tile<D>(smem + t * WarpStage<D>::BYTES, &full[t], &tmK, &tmV, g, rc.s_begin + t * kWarpTile,
+                         pol);
+  }
+  WarpTileState<KT, D, NH> st;
+  st.reset();
+  st.init_offsets(lane);
+  st.load_q(p, r, g * p.G, lane);
+
+  int consumed = 0;
+  bool aborted = false;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int stg = t % NS;
+    if (!mbar_wait_bounded(&full[stg], (t / NS) & 1, p.status)) {
+      aborted = true;
+      break;
     }
+    unsigned char* stage = smem + stg * WarpStage<D>::BYTES;
+    st.load_tile(stage);
+    consumed = t + 1;
+    auto refill = [&]() {
+      __syncwarp();
+      if (lane == 0 && t + NS < n_tiles) {
+        // the lanes' shared-memory reads of this stage precede its async refill
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_warp_tile<D>(stage, &full[stg], &tmK, &tmV, g, rc.s_begin + (t + NS) * kWarpTile, pol);
+      }
+    };
+    if (decltype(st)::kEarlyRelease) refill();
+    st.compute(p, rc, r, rc.s_begin + t * kWarpTile, has_filter, lane, stage);
+    if (!decltype(st)::kEarlyRelease) refill();
   }
-#pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int d = lane + 32 * i;
-    if (d < p.D) store_from_float(p.out.out, obase + d, p.out.type, O[i] / L);
+  if (aborted) {
+    // leave no copy in flight: wait (bounded) for every issued, unconsumed tile
+    if (lane == 0)
+      for (int t = consumed; t < min(n_tiles, consumed + NS); ++t)
+        mbar_wait_bounded(&full[t % NS], (t / NS) & 1, nullptr);
+    __syncwarp();
   }
+  st.finish_sums();
+  if (p.S == 1)
+    st.write_final(p, r, g * p.G, lane, aborted);
+  else
+    st.write_partial(p.part.o, p.part.ml, ((int64_t)r * p.Hkv + g) * p.S + s, p.G, lane, aborted);
 }
 
 template <typename KT, int D, int HPW, int HG>
@@ -444,6 +467,32 @@ cudaError_t launch_decode_t(const DecodePlan& p, const CUtensorMap& tmK, const C
   const int threads = 32 * (kKeyWarps * HG + 1);
   kern<<<dim3((unsigned)blocks), threads, Sm::kTotal, stream>>>(tmK, tmV, p);
   return cudaGetLastError();
+}
+
+template <typename KT, int D, int NH>
+cudaError_t launch_decode_mma_t(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                cudaStream_t stream) {
+  auto kern = decode_warp_kernel<KT, D, NH>;
+  static std::atomic<unsigned long long> smem_set{0ull};
+  cudaError_t e = set_smem_limit_once(smem_set, kern, WarpRing<D>::TOTAL);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (int64_t)p.R * p.Hkv * p.S;
+  kern<<<dim3((unsigned)blocks), 32, WarpRing<D>::TOTAL, stream>>>(tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+template <typename KT>
+cudaError_t launch_decode_mma(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                              cudaStream_t stream) {
+  const bool h16 = p.G > 8;
+  switch (p.D) {
+    case 64: return h16 ? launch_decode_mma_t<KT, 64, 16>(p, tmK, tmV, stream)
+                        : launch_decode_mma_t<KT, 64, 8>(p, tmK, tmV, stream);
+    case 128: return h16 ? launch_decode_mma_t<KT, 128, 16>(p, tmK, tmV, stream)
+                         : launch_decode_mma_t<KT, 128, 8>(p, tmK, tmV, stream);
+    default: return h16 ? launch_decode_mma_t<KT, 256, 16>(p, tmK, tmV, stream)
+                        : launch_decode_mma_t<KT, 256, 8>(p, tmK, tmV, stream);
+  }
 }
 
 template <typename KT, int D>
@@ -470,35 +519,29 @@ cudaError_t launch_decode_k(const DecodePlan& p, const CUtensorMap& tmK, const C
 
 }  // namespace
 
+bool decode_uses_mma(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh) {
+  // Q must already be in the cache dtype (no extra rounding) and its pairs of
+  // elements 4-byte aligned for the A-fragment loads.
+  return (kv_type == ATTN_F16 || kv_type == ATTN_BF16) && q_type == kv_type &&
+         (reinterpret_cast<uintptr_t>(q) & 3u) == 0 && (q_sr % 2) == 0 && (q_sh % 2) == 0;
+}
+
 bool decode_shape_supported(int kv_type, int D, int G) {
   return (kv_type == ATTN_F32 || kv_type == ATTN_F16 || kv_type == ATTN_BF16) &&
          (D == 64 || D == 128 || D == 256) && G >= 1 && G <= 16;
 }
 
-cudaError_t launch_decode(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                          cudaStream_t stream) {
+cudaError_t launch_decode_slices(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                 cudaStream_t stream) {
+  if (p.mma) {
+    if (p.kv_type == ATTN_F16) return launch_decode_mma<__half>(p, tmK, tmV, stream);
+    return launch_decode_mma<__nv_bfloat16>(p, tmK, tmV, stream);
+  }
   switch (p.kv_type) {
     case ATTN_F32: return launch_decode_k<float>(p, tmK, tmV, stream);
     case ATTN_F16: return launch_decode_k<__half>(p, tmK, tmV, stream);
     default: return launch_decode_k<__nv_bfloat16>(p, tmK, tmV, stream);
   }
-}
-
-cudaError_t launch_split_k_reduce(const ReducePlan& p, cudaStream_t stream) {
-  const int64_t warps = (int64_t)p.R * p.Hq;
-  const int threads = 256;
-  const int64_t blocks = (warps * 32 + threads - 1) / threads;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)blocks);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = p.use_pdl ? 1 : 0;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, split_k_reduce_kernel, p);
 }
 
 }  // namespace attn

@@ -1,0 +1,314 @@
+// decode_stream.cu -- balanced persistent split-K decode for 16-bit caches
+// (attn_decode with n_slices == 0 and Q in the cache dtype).
+//
+// The split-K idea of the pages (TensorFold PR #2595: split each row's keys
+// into slices, fold the slice partials afterwards) with slices sized for the
+// GPU instead of for the row: flatten every (row, KV head) pair's cells into
+// 16-cell tiles, pair after pair, and give each of W resident warps
+// (W = SMs x warps per SM) an equal contiguous run of that tile space.  A warp
+// streams its run through one TMA ring without restarting at pair
+// boundaries, folds it with the tensor-core tile step of decode_tile.cuh, and
+// writes one partial record per pair it touches.  Every warp gets the same
+// number of tiles (+-1), whatever the mix of row lengths, so no SM idles at
+// the end of the launch.
+//
+// Record slots, with no prefix sums in the combine: the warp in which a pair
+// STARTS writes the pair's "home" slot W + pair; any later warp that covers
+// part of the pair covers it from the start of its own run, so it writes its
+// own slot w (a run can start inside at most one pair).  The combine walks a
+// pair's home slot, then the slots of the following warps up to the one that
+// holds the pair's last tile, in tile order, so the result is deterministic.
+//
+// A planner kernel first writes row_tiles[r] (exclusive prefix of each row's
+// tile count); the persistent kernel and the combine run behind it with
+// programmatic dependent launch.
+#include "common.cuh"
+#include "decode_tile.cuh"
+#include "internal.h"
+#include "mma.cuh"
+
+namespace attn {
+
+namespace {
+
+template <int D>
+struct StreamRing {
+  static constexpr int NS = (D <= 128) ? 3 : 2;      // ring stages per warp
+  static constexpr int BAR_OFF = NS * WarpStage<D>::BYTES;
+  static constexpr int TOTAL = BAR_OFF + NS * 8 + 1024;   // + alignment slack for the swizzle
+};
+
+__device__ __forceinline__ int64_t row_len(const DecodePlan& p, int r) {
+  int32_t b = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
+  int32_t e = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
+  b = max(b, 0);
+  e = min(e, p.N);
+  return e > b ? (int64_t)e - b : 0;
+}
+
+// row_tiles[r] = sum over r' < r of ceil(len_r' / 16); row_tiles[R] = total.
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodePlan p) {
+  pdl_launch_dependents();
+  __shared__ long long wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  long long carry = 0;
+  for (int base = 0; base < p.R; base += 1024) {
+    const int r = base + tid;
+    const long long n = r < p.R ? (row_len(p, r) + kWarpTile - 1) / kWarpTile : 0;
+    long long x = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      long long v = wsum[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
+      }
+      wsum[lane] = v;
+    }
+    __syncthreads();
+    const long long excl = x - n + (wid > 0 ? wsum[wid - 1] : 0);
+    if (r < p.R) p.row_tiles[r] = carry + excl;
+    carry += wsum[31];
+    __syncthreads();
+  }
+  if (tid == 0) p.row_tiles[p.R] = carry;
+}
+
+// Position in the flattened tile space: row r, KV head g, tile j of nt.
+struct Cursor {
+  int r, g;
+  int64_t j, nt;
+  int32_t begin, end;
+};
+
+__device__ __forceinline__ void cursor_load_row(const DecodePlan& p, Cursor& c) {
+  c.nt = p.row_tiles[c.r + 1] - p.row_tiles[c.r];
+  int32_t b = p.f.row_begin ? __ldg(p.f.row_begin + c.r) : 0;
+  int32_t e = p.f.row_end ? __ldg(p.f.row_end + c.r) : p.N;
+  b = max(b, 0);
+  e = min(e, p.N);
+  c.begin = b;
+  c.end = max(e, b);
+}
+
+// Move to the next tile; rows without tiles are skipped.
+__device__ __forceinline__ void cursor_next(const DecodePlan& p, Cursor& c) {
+  if (++c.j < c.nt) return;
+  c.j = 0;
+  if (++c.g < p.Hkv) return;
+  c.g = 0;
+  do {
+    ++c.r;
+    cursor_load_row(p, c);
+  } while (c.nt == 0 && c.r + 1 < p.R);
+}
+
+template <typename KT, int D, int NH>
+__global__ void __launch_bounds__(32)
+decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const DecodePlan p) {
+  constexpr int NS = StreamRing<D>::NS;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + StreamRing<D>::BAR_OFF);
+  const int lane = threadIdx.x;
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();   // row_tiles from the planner
+
+  const int64_t W = p.W, Hkv = p.Hkv;
+  const int64_t T = Hkv * p.row_tiles[p.R];
+  const int64_t w = p.grid_order ? W - 1 - blockIdx.x : blockIdx.x;
+  const int64_t t0 = T * w / W, t1 = T * (w + 1) / W;
+  if (t0 >= t1) return;
+
+  // the row holding tile t0: the last r with Hkv * row_tiles[r] <= t0
+  // (32-ary search: each round the lanes probe 32 evenly spaced rows)
+  int lo = 0, hi = p.R;   // answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int64_t span = hi - lo;
+    const int64_t step = (span + 31) / 32;
+    const int64_t probe = lo + lane * step;
+    const bool ok = probe < hi && Hkv * p.row_tiles[probe] <= t0;
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    const int k = 31 - __clz(m);       // lane 0 always qualifies (row_tiles[lo] <= t0)
+    lo = (int)(lo + k * step);
+    hi = (int)((int64_t)hi < lo + step ? (int64_t)hi : lo + step);
+  }
+  Cursor c;
+  c.r = lo;
+  cursor_load_row(p, c);
+  {
+    const int64_t off = t0 - Hkv * p.row_tiles[c.r];
+    c.g = (int)(off / c.nt);
+    c.j = off % c.nt;
+  }
+  Cursor ic = c;   // issue cursor (lane 0 runs it NS tiles ahead)
+  const int64_t n = t1 - t0;
+  uint64_t pol = 0;
+  int64_t issued = 0;
+  // The issue cursor only advances right before issuing a tile that exists,
+  // so it never moves past the last tile of the run.
+  if (lane == 0) {
+    pol = policy_evict_first();
+    for (; issued < (n < NS ? n : (int64_t)NS); ++issued) {
+      if (issued > 0) cursor_next(p, ic);
+      issue_warp_tile<D>(smem + issued * WarpStage<D>::BYTES, &full[issued], &tmK, &tmV, ic.g,
+                         ic.begin + (int)(ic.j * kWarpTile), pol);
+    }
+  }
+
+  const bool has_filter = (p.f.cell_seq && p.f.row_seq) || p.f.causal || p.f.mask;
+  auto make_ctx = [&](const Cursor& cc) {
+    RowCtx rc;
+    rc.begin = cc.begin;
+    rc.end = cc.end;
+    rc.s_begin = cc.begin;
+    rc.s_end = cc.end;
+    rc.row_seq = p.f.row_seq ? __ldg(p.f.row_seq + cc.r) : 0;
+    rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + cc.r) : (int64_t)(cc.end - cc.begin - 1);
+    return rc;
+  };
+  RowCtx rc = make_ctx(c);
+  WarpTileState<KT, D, NH> st;
+  st.reset();
+  st.init_offsets(lane);
+  st.load_q(p, c.r, c.g * p.G, lane);
+
+  bool aborted = false;
+  int64_t k = 0;
+  for (; k < n; ++k) {
+    const int stg = (int)(k % NS);
+    if (!mbar_wait_bounded(&full[stg], (uint32_t)((k / NS) & 1), p.status)) {
+      aborted = true;
+      break;
+    }
+    unsigned char* stage = smem + stg * WarpStage<D>::BYTES;
+    st.load_tile(stage);
+    auto refill = [&]() {
+      __syncwarp();
+      if (lane == 0 && issued < n) {
+        // the lanes' shared-memory reads of this stage precede its async refill
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        cursor_next(p, ic);
+        issue_warp_tile<D>(stage, &full[stg], &tmK, &tmV, ic.g, ic.begin + (int)(ic.j * kWarpTile), pol);
+        ++issued;
+      }
+    };
+    if (decltype(st)::kEarlyRelease) refill();
+    st.compute(p, rc, c.r, c.begin + (int)(c.j * kWarpTile), has_filter, lane, stage);
+    if (!decltype(st)::kEarlyRelease) refill();
+    const bool last = (k + 1 == n);
+    if (c.j + 1 == c.nt || last) {
+      // the pair ends here (or this warp's run does): emit its record
+      st.finish_sums();
+      const int64_t pair = (int64_t)c.r * Hkv + c.g;
+      const int64_t pair_start = Hkv * p.row_tiles[c.r] + (int64_t)c.g * c.nt;
+      const int64_t slot = pair_start >= t0 ? W + pair : w;
+      st.write_partial(p.part.o, p.part.ml, slot, p.G, lane, false);
+      if (!last) {
+        cursor_next(p, c);
+        rc = make_ctx(c);
+        st.reset();
+        st.load_q(p, c.r, c.g * p.G, lane);
+      }
+    } else {
+      ++c.j;
+    }
+  }
+  if (aborted) {
+    // poison the record in progress and leave no copy in flight
+    const int64_t pair = (int64_t)c.r * Hkv + c.g;
+    const int64_t pair_start = Hkv * p.row_tiles[c.r] + (int64_t)c.g * c.nt;
+    st.write_partial(p.part.o, p.part.ml, pair_start >= t0 ? W + pair : w, p.G, lane, true);
+    if (lane == 0)
+      for (int64_t kk = k; kk < issued; ++kk) mbar_wait_bounded(&full[kk % NS], (uint32_t)((kk / NS) & 1), nullptr);
+    __syncwarp();
+  }
+}
+
+template <typename KT, int D, int NH>
+cudaError_t launch_stream_t(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            cudaStream_t stream, cudaEvent_t after_main) {
+  auto kern = decode_stream_kernel<KT, D, NH>;
+  static std::atomic<unsigned long long> smem_set{0ull};
+  cudaError_t e = set_smem_limit_once(smem_set, kern, StreamRing<D>::TOTAL);
+  if (e != cudaSuccess) return e;
+  decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.W);
+  cfg.blockDim = dim3(32);
+  cfg.dynamicSmemBytes = StreamRing<D>::TOTAL;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmK, tmV, p);
+  if (e != cudaSuccess) return e;
+  if (after_main) cudaEventRecord(after_main, stream);
+  return cudaSuccess;
+}
+
+template <typename KT>
+cudaError_t launch_stream_k(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            cudaStream_t stream, cudaEvent_t ev) {
+  const bool h16 = p.G > 8;
+  switch (p.D) {
+    case 64: return h16 ? launch_stream_t<KT, 64, 16>(p, tmK, tmV, stream, ev)
+                        : launch_stream_t<KT, 64, 8>(p, tmK, tmV, stream, ev);
+    case 128: return h16 ? launch_stream_t<KT, 128, 16>(p, tmK, tmV, stream, ev)
+                         : launch_stream_t<KT, 128, 8>(p, tmK, tmV, stream, ev);
+    default: return h16 ? launch_stream_t<KT, 256, 16>(p, tmK, tmV, stream, ev)
+                        : launch_stream_t<KT, 256, 8>(p, tmK, tmV, stream, ev);
+  }
+}
+
+template <typename KT, int D, int NH>
+int stream_blocks_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<KT, D, NH>, 32,
+                                                    StreamRing<D>::TOTAL) != cudaSuccess || n <= 0) {
+    // no device: the shared-memory bound of a 228 KB SM with 1 KB reserved per CTA
+    n = (228 * 1024) / (StreamRing<D>::TOTAL + 1024);
+  }
+  return n;
+}
+
+}  // namespace
+
+int decode_stream_warps(int kv_type, int D, int G, int sms) {
+  int per_sm;
+  const bool h16 = G > 8;
+  if (kv_type == ATTN_F16) {
+    per_sm = D == 64 ? (h16 ? stream_blocks_per_sm<__half, 64, 16>() : stream_blocks_per_sm<__half, 64, 8>())
+           : D == 128 ? (h16 ? stream_blocks_per_sm<__half, 128, 16>() : stream_blocks_per_sm<__half, 128, 8>())
+                      : (h16 ? stream_blocks_per_sm<__half, 256, 16>() : stream_blocks_per_sm<__half, 256, 8>());
+  } else {
+    per_sm = D == 64 ? (h16 ? stream_blocks_per_sm<__nv_bfloat16, 64, 16>() : stream_blocks_per_sm<__nv_bfloat16, 64, 8>())
+           : D == 128 ? (h16 ? stream_blocks_per_sm<__nv_bfloat16, 128, 16>() : stream_blocks_per_sm<__nv_bfloat16, 128, 8>())
+                      : (h16 ? stream_blocks_per_sm<__nv_bfloat16, 256, 16>() : stream_blocks_per_sm<__nv_bfloat16, 256, 8>());
+  }
+  return std::max(1, per_sm) * std::max(1, sms);
+}
+
+cudaError_t launch_decode_stream(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                 cudaStream_t stream, cudaEvent_t after_main) {
+  if (p.kv_type == ATTN_F16) return launch_stream_k<__half>(p, tmK, tmV, stream, after_main);
+  return launch_stream_k<__nv_bfloat16>(p, tmK, tmV, stream, after_main);
+}
+
+}  // namespace attn

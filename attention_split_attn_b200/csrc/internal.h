@@ -1,5 +1,5 @@
 // internal.h -- host-side plans handed from the C-ABI layer (api.cu) to the
-// kernel launchers (decode.cu, selected.cu, prefill.cu).  Not installed.
+// kernel launchers.  Not installed.
 #pragma once
 
 #include <cuda.h>
@@ -25,7 +25,6 @@ struct Logits {
   const float* sinks;
 };
 
-// Output of a row: where and in which dtype.
 struct OutSpec {
   void* out;
   int32_t type;
@@ -38,12 +37,13 @@ struct QSpec {
   int64_t sr, sh;
 };
 
-// Split-K partial store: per (row, q head, slice) the slice's running max m
-// and sum l (natural-log domain) and its unnormalised output o[D].
+// Split partials: one record per (slot, q head of the KV group): the running
+// max m and sum l (natural-log domain) and the unnormalised output o[D].
+// Records are laid out [slot][G][D] (o) and [slot][G][2] (ml).
 struct Partials {
-  float* o;    // [R][Hq][S][D]
-  float* ml;   // [R][Hq][S][2]
-  int32_t S;
+  float* o;
+  float* ml;
+  int32_t S;   // slice scheme: slices per (row, KV head); slot = (r*Hkv + g)*S + s
 };
 
 // ---- decode ----------------------------------------------------------------
@@ -53,34 +53,47 @@ struct DecodePlan {
   OutSpec out;
   RowFilter f;
   Logits lg;
-  int32_t S;          // slices per row (grid extent)
-  int32_t C;          // cells per slice (multiple of 32); the last slice takes the rest
-  int32_t grid_order; // 0 rows fastest, 1 slices fastest
-  Partials part;      // used when S > 1
+  int32_t S;          // slice scheme: slices per row (grid extent)
+  int32_t C;          // slice scheme: cells per slice (multiple of 32); the last slice takes the rest
+  int32_t grid_order; // 0: natural order; 1: reversed / slices fastest (results identical)
+  Partials part;      // used when S > 1 or in the balanced scheme
   int* status;
   int32_t kv_type;
-  int32_t hpw, hg;    // q heads per warp (padded) and head groups
+  int32_t hpw, hg;    // CUDA-core kernel: q heads per warp (padded) and head groups
+  int32_t mma;        // 1: tensor-core kernels (16-bit cache, Q in the cache dtype)
+  // balanced persistent scheme (n_slices == 0 with the tensor-core kernels):
+  int32_t W;          // warps of the persistent grid
+  int64_t* row_tiles; // [R+1] exclusive prefix of 16-cell tiles per row (planner output)
 };
 
+bool decode_uses_mma(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh);
 bool decode_shape_supported(int kv_type, int D, int G);
-cudaError_t launch_decode(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                          cudaStream_t stream);
 
-// split_k_reduce over decode partials (also used by the selected op).  Reads
-// n_used(r) slices for row r: n_used = 0 if empty else min(S, ceil(len/C)),
-// with len from `f` (decode) or from `counts` (selected: per-row list length).
-struct ReducePlan {
-  int32_t R, Hq, D;
+// (rows, heads, slices) grid: one CTA per unit; split_k combine when S > 1.
+cudaError_t launch_decode_slices(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                 cudaStream_t stream);
+
+// Balanced persistent scheme: planner kernel, then W single-warp CTAs that
+// each take an equal run of the flattened (row, KV head, 16-cell tile) space.
+int decode_stream_warps(int kv_type, int D, int G, int sms);
+cudaError_t launch_decode_stream(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                 cudaStream_t stream, cudaEvent_t after_main);
+
+// ---- combine (split_k_reduce) -------------------------------------------------
+// Folds the partial records of each (row, q head) in slot order with the sink.
+struct CombinePlan {
+  int32_t R, Hq, Hkv, G, D;
   OutSpec out;
   const float* sinks;
   Partials part;
-  // slice count per row: either from ranges (row_begin/row_end, C) or a
-  // device array of counts (n_used per row)
-  const int32_t *row_begin, *row_end;
+  int32_t mode;                          // 0: slice scheme, 1: balanced scheme
+  const int32_t *row_begin, *row_end;    // slice scheme: n_used(r) from ranges ...
   int32_t N, C;
-  const int32_t* n_used;  // if non-NULL, overrides the range rule
+  const int32_t* n_used;                 // ... or from per-row counts (selected op)
+  const int64_t* row_tiles;              // balanced scheme
+  int32_t W;
   int use_pdl;
 };
-cudaError_t launch_split_k_reduce(const ReducePlan& p, cudaStream_t stream);
+cudaError_t launch_combine(const CombinePlan& p, cudaStream_t stream);
 
 }  // namespace attn

@@ -1,0 +1,353 @@
+"""Benchmark of attention over a KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: GQA split-K decode -- 16 sequences x 1 query row, 32 query heads over
+8 KV heads, head_dim 128, bf16 KV cache [16 x 8192 cells, 8, 128] with
+per-sequence lengths uniform in [1024, 8192] (seed 1002), bf16 output, slice
+count from the planner.  One step = one attn_decode call (slice kernel +
+split_k_reduce) over one batch.  The metric is attention GB/s: the algorithmic
+bytes of a step (K and V rows of every visible cell, Q and the output) over
+the step time, with the HBM roofline of the dominant kernel beside it.
+
+Timing: W untimed warm-up steps, then K steps between a barrier and a device
+synchronize, timed with CUDA events on the launching stream, max over ranks.
+Each step reads a different one of three resident input sets (~0.9 GB of K/V
+in all), so a step never finds the previous step's cache in L2 (126 MB).
+
+--impl reference times the FP64 CPU oracle on the host cores on a bounded
+sample of the same workload (the pages ship no code; the oracle is the
+baseline arm).  Under torchrun every rank runs its own batch (weak scaling;
+the path has no collective); only a scalar max of the step time crosses ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import attention_split_attn_b200 as A                      # noqa: E402
+from attention_split_attn_b200 import workloads as W       # noqa: E402
+
+METRIC = "attention GB/s (decode, % HBM peak); prefill TFLOP/s (% bf16 tensor peak)"
+WORKLOAD = "gqa_decode: 16 seq x 1 row, Hq 32 / Hkv 8, D 128, bf16 KV, len U[1024,8192], bf16 out"
+N_SETS = 3
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws == 1:
+        return 0, 1, 0
+    import torch.distributed as dist
+    import datetime
+    rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, ws, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_bytes(p) -> int:
+    """K and V rows of every visible cell for its KV head, plus Q and out."""
+    lens = (p.row_end - p.row_begin).to(torch.int64)
+    kv = int(lens.sum()) * p.n_head_kv * p.head_dim * p.k.element_size() * 2
+    q = p.q.numel() * p.q.element_size()
+    o = p.n_rows * p.n_head_q * p.head_dim * torch.empty((), dtype=p.out_dtype).element_size()
+    return kv + q + o
+
+
+def run_reference(args, rank, world):
+    """The FP64 oracle on the host cores, on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    p = W.gqa_decode(poison_unused=False)
+    rows = [0, 1]                       # a bounded sample: 2 of the 16 rows
+    sub = p.row_subset(rows)
+    bytes_per_step = algorithmic_bytes(sub)
+    cores = os.cpu_count() or 1
+    prep = oracle.Prepared(sub)
+    for _ in range(max(0, args.warmup)):
+        prep.run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        prep.run()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    gbs = bytes_per_step / dt / 1e9
+    line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": "rows 0-1 of 16", "parallelism": "host threads"},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": min(cores, len(rows)),
+                             "kind": "oracle", "sample": "rows 0-1 of the 16-row batch (one thread per row)"},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline():
+    """Oracle throughput on the host cores over the whole 16-row batch, repeated
+    for about 10 s."""
+    import oracle
+    p = W.gqa_decode(poison_unused=False)
+    nbytes = algorithmic_bytes(p)
+    cores = os.cpu_count() or 1
+    prep = oracle.Prepared(p)
+    prep.run(n_threads=cores)
+    t0, n = time.perf_counter(), 0
+    while True:
+        prep.run(n_threads=cores)
+        n += 1
+        if time.perf_counter() - t0 > 10.0:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": min(cores, p.n_rows), "kind": "oracle",
+            "sample": f"the full 16-row batch, {n} repetitions (~10 s), one thread per row"}
+
+
+def run_ours(args, rank, world, local):
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    A.load_library()
+    hbm_peak, _, peak_kind = _peaks()
+
+    # three resident input sets of the same shape (different seeds per set and rank)
+    sets = []
+    for i in range(N_SETS):
+        p = W.gqa_decode(seed=1002 + 7919 * rank + 104729 * i, poison_unused=False)
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+        sets.append(dict(p=p, args=a, ws=ws, keep=(q, k, v, out, kw), bytes=algorithmic_bytes(p)))
+    S = A.workspace_size(sets[0]["args"], A.OP_DECODE)   # nonzero -> split
+    launches_per_step = 2 if S > 0 else 1
+
+    # a quick parity spot check outside the timed region (2 rows vs the oracle)
+    if rank == 0:
+        import oracle
+        A.attn_decode_args(sets[0]["args"], ws=sets[0]["ws"])
+        torch.cuda.synchronize()
+        out = sets[0]["keep"][3][:2].double().cpu().numpy()
+        ref = oracle.attn(sets[0]["p"].row_subset([0, 1]))
+        nmse = float(((out - ref) ** 2).sum() / (ref ** 2).sum())
+        assert nmse < 1e-5, f"parity spot check failed: NMSE {nmse}"
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        st = sets[i % N_SETS]
+        A.attn_decode_args(st["args"], ws=st["ws"])
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)          # torch creates the handle on first record; the library re-records it
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total_bytes = 0
+    with Clocks(local) as clk:
+        _barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            st = sets[i % N_SETS]
+            A.attn_decode_timed_args(st["args"], st["ws"], ev[i], stream=stream)
+            total_bytes += st["bytes"]
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        _barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = _max_over_ranks(elapsed_ms, world)
+    main_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    step_bytes = total_bytes / args.steps
+    value = step_bytes * world * args.steps / (elapsed_ms * 1e-3) / 1e9
+
+    # dominant kernel: the slice kernel (events[0] -> events[1])
+    kmean_ms = sum(main_ms) / len(main_ms)
+    achieved = step_bytes / (kmean_ms * 1e-3) / 1e9
+    traffic = _recorded_traffic()
+
+    e2e = run_e2e(args, sets, stream)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows_per_step": 16 * world, "slices": "planner",
+                   "l2": "3 rotating input sets, each step's K/V (302 MB) larger than L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "rows_per_s": 16 * world * args.steps / (elapsed_ms * 1e-3),
+        "frac_of_hbm_peak": value / world / hbm_peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "kernel": "decode_slice_kernel", "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _recorded_traffic():
+    """DRAM bytes per launch of the slice kernel from the committed ncu summary,
+    if it was taken on the current kernel build (else null)."""
+    path = os.path.join(ROOT, "profiles", "decode_slice_kernel_gqa_decode.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "attention_split_attn_b200", "csrc", "decode.cu")
+    import hashlib
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d.get("dram_bytes_per_launch") if d.get("decode_cu_sha256_16") == h else None
+
+
+def run_e2e(args, sets, stream):
+    """The same step through the C ABI from pinned HOST buffers: every step
+    copies its inputs (Q, the K/V rows each sequence uses, row ranges) to the
+    device, runs attn_decode, and reads the output back."""
+    st0 = sets[0]
+    p = st0["p"]
+    q, k, v, out, kw = st0["keep"]
+    b = p.row_begin.tolist()
+    e = p.row_end.tolist()
+    host = {"q": p.q.pin_memory(), "rb": p.row_begin.pin_memory(), "re": p.row_end.pin_memory(),
+            "out": torch.empty(out.shape, dtype=out.dtype).pin_memory()}
+    host_k = [p.k[b[i]:e[i]].contiguous().pin_memory() for i in range(len(b))]
+    host_v = [p.v[b[i]:e[i]].contiguous().pin_memory() for i in range(len(b))]
+    h2d = (host["q"].numel() * host["q"].element_size() + 2 * host["rb"].numel() * 4
+           + sum(t.numel() * t.element_size() for t in host_k + host_v))
+    d2h = host["out"].numel() * host["out"].element_size()
+
+    def step():
+        q.copy_(host["q"], non_blocking=True)
+        kw["row_begin"].copy_(host["rb"], non_blocking=True)
+        kw["row_end"].copy_(host["re"], non_blocking=True)
+        for i in range(len(b)):
+            k[b[i]:e[i]].copy_(host_k[i], non_blocking=True)
+            v[b[i]:e[i]].copy_(host_v[i], non_blocking=True)
+        A.attn_decode_args(st0["args"], ws=st0["ws"])
+        host["out"].copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(n):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    return {"value": st0["bytes"] / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    rank, world, local = _dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

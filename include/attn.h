@@ -153,6 +153,14 @@ int32_t attn_decode(const attn_args *args, void *ws, size_t ws_bytes, void *stre
 int32_t attn_selected(const attn_selected_args *args, void *ws, size_t ws_bytes, void *stream);
 int32_t attn_prefill(const attn_args *args, void *ws, size_t ws_bytes, void *stream);
 
+/* Timing hooks: the same operations, and additionally cudaEventRecord of
+ * events[0] before the first kernel, events[1] right after the main kernel
+ * (decode: the slice kernel; selected: the gather kernel; prefill: the
+ * tensor-core kernel) and events[2] after the last kernel, all on `stream`.
+ * Each entry is a cudaEvent_t passed as void*, or NULL to skip it.          */
+int32_t attn_decode_timed(const attn_args *args, void *ws, size_t ws_bytes, void *stream,
+                          void *const events[3]);
+
 /* Synchronizes `stream`, then reads and clears the device status word on the
  * current device: ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on
  * a bounded wait since the last check.                                      */

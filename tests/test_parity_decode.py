@@ -171,3 +171,39 @@ def test_workspace_too_small_is_refused(cuda_lib):
     st = lib.attn_decode(ctypes.byref(args), ws.data_ptr(), ws.numel(),
                          torch.cuda.current_stream().cuda_stream)
     assert st == -3
+
+
+# ---- the balanced persistent scheme (n_slices = 0, 16-bit cache) -----------
+
+def test_balanced_semantics_sweep(cuda_lib, semantics_problem):
+    p, ref = semantics_problem
+    check(p, run_decode(p, n_slices=0), "semantics balanced", ref=ref)
+
+
+def test_balanced_order_bit_identical(cuda_lib):
+    """Reversing which warp takes which run changes nothing, bit for bit."""
+    p = W.gqa_decode(n_seq=8, cap=4096)
+    a = run_decode(p, n_slices=0)
+    b = run_decode(p, n_slices=0, grid_order=1)
+    c = run_decode(p, n_slices=0)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+    check(p, a, "gqa_decode balanced")
+
+
+def test_balanced_one_long_row(cuda_lib):
+    """One row whose cells are spread over every resident warp (hundreds of
+    records per row in the combine)."""
+    p = W.random_problem(77, R=1, Hq=4, Hkv=1, D=128, N=120000, kv_dtype=torch.bfloat16,
+                         out_dtype=torch.float32, ranges=False, sinks=True)
+    check(p, run_decode(p, n_slices=0), "one long row")
+
+
+def test_balanced_more_warps_than_tiles(cuda_lib):
+    """Fewer tiles than warps: most warp runs are empty."""
+    p = W.random_problem(78, R=3, Hq=8, Hkv=2, D=64, N=40, kv_dtype=torch.float16,
+                         out_dtype=torch.float16, lengths=[40, 17, 0], sinks=True)
+    check(p, run_decode(p, n_slices=0), "tiny balanced")
+    p = W.random_problem(79, R=70, Hq=16, Hkv=1, D=256, N=300, kv_dtype=torch.bfloat16,
+                         out_dtype=torch.float32, softcap=3.0)
+    check(p, run_decode(p, n_slices=0), "many short rows")
