@@ -31,8 +31,8 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
-           "attn_prefill", "attn_decode_timed", "attn_check_device_status", "attn_strerror",
-           "attn_last_error", "attn_abi_version")
+           "attn_prefill", "attn_decode_timed", "attn_decode_noalloc", "attn_check_device_status",
+           "attn_strerror", "attn_last_error", "attn_abi_version")
 
 
 class AttnArgs(ctypes.Structure):
@@ -97,6 +97,8 @@ def load_library():
             lib.attn_decode_timed.restype = ctypes.c_int32
             lib.attn_decode_timed.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t,
                                               ctypes.c_void_p, ctypes.c_void_p * 3]
+            lib.attn_decode_noalloc.restype = ctypes.c_int32
+            lib.attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
             lib.attn_selected.restype = ctypes.c_int32
             lib.attn_selected.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
                                           ctypes.c_size_t, ctypes.c_void_p]

@@ -268,6 +268,10 @@ int32_t check_decode(const attn_args* a) {
 }  // namespace
 }  // namespace attn
 
+namespace attn {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace attn
+
 using namespace attn;
 
 extern "C" {

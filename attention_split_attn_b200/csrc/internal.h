@@ -96,4 +96,7 @@ struct CombinePlan {
 };
 cudaError_t launch_combine(const CombinePlan& p, cudaStream_t stream);
 
+// Set the message attn_last_error() returns on this thread.
+void set_last_error(const char* msg);
+
 }  // namespace attn

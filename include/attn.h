@@ -161,6 +161,22 @@ int32_t attn_prefill(const attn_args *args, void *ws, size_t ws_bytes, void *str
 int32_t attn_decode_timed(const attn_args *args, void *ws, size_t ws_bytes, void *stream,
                           void *const events[3]);
 
+/* attn_decode for callers that cannot allocate device memory (a real-time
+ * loop that must not block in an allocator, a plugin with no memory pool of
+ * its own, code that only receives pointers to its inputs and outputs).  The
+ * pages have no counterpart: this is a convenience of this library.
+ * Arguments and results are those of attn_decode; the split partials live in
+ * one built-in 16 MiB device array per GPU (held until the process exits)
+ * instead of a caller workspace, and nothing is allocated per call.
+ *  - A problem needing more scratch than that returns ATTN_ERR_WORKSPACE
+ *    (attn_last_error() gives the size); nothing is launched.
+ *  - All calls share the array: calls that may overlap on the GPU race and
+ *    corrupt each other; issue them in order on one stream.  Nothing in the
+ *    array needs to start at zero.
+ *  - The first call on each device looks up the array's address
+ *    (cudaGetSymbolAddress, no allocation); make it before any stream capture. */
+int32_t attn_decode_noalloc(const attn_args *args, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word on the
  * current device: ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on
  * a bounded wait since the last check.                                      */
