@@ -33,7 +33,7 @@ namespace {
 
 template <int D>
 struct StreamRing {
-  static constexpr int NS = (D <= 128) ? 3 : 2;      // ring stages per warp
+  static constexpr int NS = 2;                       // ring stages per warp
   static constexpr int BAR_OFF = NS * WarpStage<D>::BYTES;
   static constexpr int TOTAL = BAR_OFF + NS * 8 + 1024;   // + alignment slack for the swizzle
 };
