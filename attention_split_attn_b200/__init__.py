@@ -31,7 +31,8 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
-           "attn_prefill", "attn_decode_timed", "attn_decode_noalloc", "attn_check_device_status",
+           "attn_prefill", "attn_decode_timed", "attn_selected_timed", "attn_decode_noalloc",
+           "attn_check_device_status",
            "attn_strerror", "attn_last_error", "attn_abi_version")
 
 
@@ -102,6 +103,9 @@ def load_library():
             lib.attn_selected.restype = ctypes.c_int32
             lib.attn_selected.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
                                           ctypes.c_size_t, ctypes.c_void_p]
+            lib.attn_selected_timed.restype = ctypes.c_int32
+            lib.attn_selected_timed.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p * 3]
             lib.attn_check_device_status.restype = ctypes.c_int32
             lib.attn_check_device_status.argtypes = [ctypes.c_void_p]
             lib.attn_strerror.restype = ctypes.c_char_p
@@ -222,6 +226,67 @@ def decode(q, k, v, out, *, ws=None, stream=None, **kw):
     return attn_decode_args(make_args(q, k, v, out, **kw), ws=ws, stream=stream)
 
 
+def make_selected_args(q, k, v, out, sel, *, sorted_out=None, count_out=None, **kw):
+    """Fill an AttnSelectedArgs: `sel` is an int32 CUDA tensor [rows, n_sel]
+    (row stride may exceed n_sel); sorted_out [rows, n_sel] and count_out
+    [rows] are optional int32 outputs of the compaction."""
+    for key in ("row_begin", "row_end", "cell_seq", "row_seq", "mask"):
+        if kw.get(key) is not None:
+            raise ValueError(f"selected-key attention takes no {key}")
+    if kw.get("causal"):
+        raise ValueError("selected-key attention is maskless (causal must be False)")
+    a = AttnSelectedArgs()
+    a.base = make_args(q, k, v, out, **kw)
+    if sel.dtype != torch.int32 or not sel.is_cuda or sel.dim() != 2 or sel.stride(1) != 1:
+        raise ValueError("sel must be an int32 CUDA tensor [rows, n_sel] with contiguous entries")
+    a.sel, a.sel_stride_row, a.n_sel = sel.data_ptr(), sel.stride(0), sel.shape[1]
+    for name, t, shape in (("sorted_out", sorted_out, tuple(sel.shape)), ("count_out", count_out, (sel.shape[0],))):
+        if t is not None and (t.dtype != torch.int32 or not t.is_cuda or tuple(t.shape) != shape
+                              or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of shape {shape}")
+    a.sel_sorted_out = _ptr(sorted_out)
+    a.sel_count_out = _ptr(count_out)
+    return a
+
+
+def attn_selected_args(args: AttnSelectedArgs, ws: Optional[torch.Tensor] = None, stream=None):
+    """attn_selected on a prepared AttnSelectedArgs (workspace allocated if needed)."""
+    lib = load_library()
+    _raise_if(lib.attn_supports(ctypes.byref(args.base), OP_SELECTED), "attn_supports")
+    need = int(lib.attn_workspace_size(ctypes.byref(args.base), OP_SELECTED, args.n_sel))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = _workspace(need, dev, ws)
+    st = lib.attn_selected(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                           0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
+    _raise_if(st, "attn_selected")
+    return ws
+
+
+def attn_selected_timed_args(args: AttnSelectedArgs, ws: Optional[torch.Tensor], events, stream=None):
+    """attn_selected that also records three torch.cuda.Events (before the
+    compaction, after the gather kernel, after the combine)."""
+    lib = load_library()
+    handles = [None if e is None else e.cuda_event for e in events]
+    if any(h == 0 for h in handles):
+        raise ValueError("record each torch.cuda.Event once before passing it (torch creates it lazily)")
+    ev = (ctypes.c_void_p * 3)(*handles)
+    st = lib.attn_selected_timed(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                                 0 if ws is None else ws.numel() * ws.element_size(),
+                                 _stream_handle(stream), ev)
+    _raise_if(st, "attn_selected_timed")
+
+
+def selected_workspace_size(args: AttnSelectedArgs) -> int:
+    lib = load_library()
+    _raise_if(lib.attn_supports(ctypes.byref(args.base), OP_SELECTED), "attn_supports")
+    return int(lib.attn_workspace_size(ctypes.byref(args.base), OP_SELECTED, args.n_sel))
+
+
+def selected(q, k, v, out, sel, *, ws=None, stream=None, **kw):
+    """Maskless selected-key attention into `out` (see include/attn.h)."""
+    return attn_selected_args(make_selected_args(q, k, v, out, sel, **kw), ws=ws, stream=stream)
+
+
 def check_device_status(stream=None):
     lib = load_library()
     _raise_if(lib.attn_check_device_status(_stream_handle(stream)), "attn_check_device_status")
@@ -242,4 +307,8 @@ def problem_kwargs(p, device="cuda", out=None):
               row_pos=dev(p.row_pos), causal=p.causal, mask=dev(p.mask),
               alibi_slopes=dev(p.alibi_slopes), sinks=dev(p.sinks), n_slices=p.n_slices,
               max_row_len=p.max_row_len)
+    if p.sel is not None:
+        for key in ("row_begin", "row_end", "cell_seq", "row_seq", "mask", "causal", "max_row_len"):
+            kw.pop(key)
+        kw["sel"] = dev(p.sel)
     return (q, k, v, out), kw

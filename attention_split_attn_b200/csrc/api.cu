@@ -265,6 +265,65 @@ int32_t check_decode(const attn_args* a) {
   return ATTN_OK;
 }
 
+// ---- selected-key planning ---------------------------------------------------------
+constexpr int kMaxSel = 4096;
+
+int32_t check_selected_base(const attn_args* a) {
+  int32_t st = validate_common(a, ATTN_OP_SELECTED);
+  if (st != ATTN_OK) return st;
+  if (a->row_begin || a->row_end || a->cell_seq || a->row_seq || a->mask || a->causal)
+    return fail(ATTN_ERR_INVALID_ARG,
+                "selected: the op is maskless; row ranges, sequence ids, causal and mask must be unset");
+  if (a->kv_type != ATTN_F16 && a->kv_type != ATTN_BF16)
+    return fail(ATTN_ERR_UNSUPPORTED, "selected: K/V must be F16 or BF16");
+  if (a->q_type != a->kv_type) return fail(ATTN_ERR_UNSUPPORTED, "selected: Q must be in the K/V dtype");
+  if (a->n_rows > 0 && ((reinterpret_cast<uintptr_t>(a->q) & 3u) || (a->q_stride_row % 2) || (a->q_stride_head % 2)))
+    return fail(ATTN_ERR_UNSUPPORTED, "selected: Q must be 4-byte aligned with even strides");
+  return ATTN_OK;
+}
+
+struct SelShape {
+  int32_t S, C;
+};
+
+// Parts per row: one when the (row, KV head) units fill the GPU about twice
+// over, else enough parts to (the pages' rule: split rows when the grid would
+// under-fill the device), at most 64 and at most one per 32-cell block.
+SelShape plan_selected(const attn_args* a, int n_sel, int sms) {
+  SelShape s;
+  int64_t S = a->n_slices;
+  if (S == 0) {
+    const int64_t units = std::max<int64_t>(1, (int64_t)a->n_rows * a->n_head_kv);
+    const int64_t target = 4LL * std::max(sms, 1);
+    S = units >= target ? 1 : (target + units - 1) / units;
+  }
+  S = std::min<int64_t>(S, std::max<int64_t>(1, (n_sel + 31) / 32));
+  S = std::min<int64_t>(std::max<int64_t>(S, 1), 64);
+  int64_t C = (n_sel + S - 1) / S;
+  C = (C + 31) / 32 * 32;
+  s.S = (int32_t)S;
+  s.C = (int32_t)std::max<int64_t>(C, 32);
+  return s;
+}
+
+struct SelWs {
+  size_t count_off, o_off, ml_off, total;
+};
+
+SelWs selected_ws_layout(const attn_args* a, int n_sel, const SelShape& sh) {
+  SelWs w;
+  w.count_off = align256((size_t)a->n_rows * n_sel * sizeof(int32_t));
+  w.o_off = w.count_off + align256((size_t)a->n_rows * sizeof(int32_t));
+  w.ml_off = w.o_off;
+  w.total = w.o_off;
+  if (sh.S > 1) {
+    const size_t records = (size_t)a->n_rows * a->n_head_q * sh.S;
+    w.ml_off = w.o_off + align256(records * a->head_dim * sizeof(float));
+    w.total = w.ml_off + align256(records * 2 * sizeof(float));
+  }
+  return w;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -295,18 +354,21 @@ const char* attn_last_error(void) { return g_last_error.c_str(); }
 int32_t attn_supports(const attn_args* a, int32_t op) {
   switch (op) {
     case ATTN_OP_DECODE: return check_decode(a);
+    case ATTN_OP_SELECTED: return check_selected_base(a);
     default: return fail(ATTN_ERR_UNSUPPORTED, "op %d is not available in this build", op);
   }
 }
 
 size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
-  (void)n_sel;
   if (attn_supports(a, op) != ATTN_OK) return 0;
   int sms = 148;
   DeviceInfo* di = nullptr;
   if (device_info(&di) == ATTN_OK) sms = di->sms;
   switch (op) {
     case ATTN_OP_DECODE: return decode_ws_bytes(a, plan_decode(a, sms));
+    case ATTN_OP_SELECTED:
+      if (n_sel < 1 || n_sel > kMaxSel) return 0;
+      return selected_ws_layout(a, n_sel, plan_selected(a, n_sel, sms)).total;
     default: return 0;
   }
 }
@@ -404,8 +466,70 @@ int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* s
 }
 
 int32_t attn_selected(const attn_selected_args* a, void* ws, size_t ws_bytes, void* stream) {
-  (void)a; (void)ws; (void)ws_bytes; (void)stream;
-  return fail(ATTN_ERR_UNSUPPORTED, "attn_selected is not available in this build");
+  return attn_selected_timed(a, ws, ws_bytes, stream, nullptr);
+}
+
+int32_t attn_selected_timed(const attn_selected_args* a, void* ws, size_t ws_bytes, void* stream,
+                            void* const events[3]) {
+  if (!a) return fail(ATTN_ERR_INVALID_ARG, "args is NULL");
+  const attn_args* b = &a->base;
+  int32_t st = check_selected_base(b);
+  if (st != ATTN_OK) return st;
+  if (a->n_sel < 1 || a->n_sel > kMaxSel) return fail(ATTN_ERR_UNSUPPORTED, "n_sel must be 1..%d", kMaxSel);
+  if (b->n_rows == 0) return ATTN_OK;
+  if (!a->sel) return fail(ATTN_ERR_INVALID_ARG, "sel is NULL");
+  if (a->sel_stride_row < a->n_sel) return fail(ATTN_ERR_INVALID_ARG, "sel_stride_row is smaller than n_sel");
+  DeviceInfo* di = nullptr;
+  if ((st = device_info(&di)) != ATTN_OK) return st;
+  const SelShape sh = plan_selected(b, a->n_sel, di->sms);
+  const SelWs wl = selected_ws_layout(b, a->n_sel, sh);
+  if (ws == nullptr || ws_bytes < wl.total)
+    return fail(ATTN_ERR_WORKSPACE, "selected needs %zu workspace bytes, got %zu", wl.total, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(ATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const int64_t blocks = (int64_t)b->n_rows * b->n_head_kv * sh.S;
+  if (blocks > 0x7fffffffLL || b->n_rows > 0x7fffffff)
+    return fail(ATTN_ERR_UNSUPPORTED, "grid of %lld CTAs is too large", (long long)blocks);
+
+  char* wsb = static_cast<char*>(ws);
+  SelectedPlan p{};
+  p.R = b->n_rows; p.Hq = b->n_head_q; p.Hkv = b->n_head_kv; p.G = b->n_head_q / b->n_head_kv;
+  p.D = b->head_dim; p.N = b->n_cells;
+  p.q = b->q; p.q_sr = b->q_stride_row; p.q_sh = b->q_stride_head;
+  p.k = b->k; p.v = b->v; p.kv_sc = b->kv_stride_cell; p.kv_sh = b->kv_stride_head; p.kv_type = b->kv_type;
+  p.out = OutSpec{b->out, b->out_type, b->o_stride_row, b->o_stride_head};
+  p.lg = Logits{b->scale, b->softcap, b->alibi_slopes, b->sinks};
+  p.cell_pos = b->cell_pos; p.row_pos = b->row_pos;
+  p.sel = a->sel; p.sel_stride = a->sel_stride_row; p.n_sel = a->n_sel; p.n_pow2 = selected_pow2(a->n_sel);
+  p.compact = reinterpret_cast<int32_t*>(wsb);
+  p.count = reinterpret_cast<int32_t*>(wsb + wl.count_off);
+  p.sorted_out = a->sel_sorted_out; p.count_out = a->sel_count_out;
+  p.S = sh.S; p.C = sh.C;
+  if (sh.S > 1) {
+    p.part.o = reinterpret_cast<float*>(wsb + wl.o_off);
+    p.part.ml = reinterpret_cast<float*>(wsb + wl.ml_off);
+    p.part.S = sh.S;
+  }
+  p.status = di->status;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  record_event(events, 0, s);
+  cudaError_t e = launch_select_compact(p, s);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "select_compact launch: %s", cudaGetErrorString(e));
+  e = launch_selected(p, s);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "selected launch: %s", cudaGetErrorString(e));
+  record_event(events, 1, s);
+  if (sh.S > 1) {
+    CombinePlan cp{};
+    cp.R = b->n_rows; cp.Hq = b->n_head_q; cp.Hkv = b->n_head_kv; cp.G = p.G; cp.D = b->head_dim;
+    cp.out = p.out; cp.sinks = b->sinks; cp.part = p.part;
+    cp.mode = 0;
+    cp.row_len = p.count; cp.C = sh.C; cp.N = b->n_cells;
+    cp.use_pdl = (events && events[1]) ? 0 : 1;
+    e = launch_combine(cp, s);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  }
+  record_event(events, 2, s);
+  return ATTN_OK;
 }
 
 int32_t attn_prefill(const attn_args* a, void* ws, size_t ws_bytes, void* stream) {

@@ -64,6 +64,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombinePlan p) {
     int n_used;
     if (p.n_used) {
       n_used = min(__ldg(p.n_used + r), p.part.S);
+    } else if (p.row_len) {
+      const int64_t len = max(__ldg(p.row_len + r), 0);
+      n_used = len == 0 ? 0 : (int)min((int64_t)p.part.S, (len + p.C - 1) / p.C);
     } else {
       int32_t b = p.row_begin ? __ldg(p.row_begin + r) : 0;
       int32_t e = p.row_end ? __ldg(p.row_end + r) : p.N;

@@ -79,6 +79,32 @@ int decode_stream_warps(int kv_type, int D, int G, int sms);
 cudaError_t launch_decode_stream(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                  cudaStream_t stream, cudaEvent_t after_main);
 
+// ---- selected-key attention ---------------------------------------------------
+struct SelectedPlan {
+  int32_t R, Hq, Hkv, G, D, N;
+  const void* q;
+  int64_t q_sr, q_sh;
+  const void *k, *v;
+  int64_t kv_sc, kv_sh;
+  int32_t kv_type;
+  OutSpec out;
+  Logits lg;
+  const int32_t *cell_pos, *row_pos;   // ALiBi distances only
+  const int32_t* sel;                  // [R][sel_stride], first n_sel used
+  int64_t sel_stride;
+  int32_t n_sel, n_pow2;               // n_pow2: n_sel rounded up to a power of 2
+  int32_t* compact;                    // workspace [R][n_sel]: valid distinct cells, ascending
+  int32_t* count;                      // workspace [R]: their number
+  int32_t *sorted_out, *count_out;     // caller's optional copies (or NULL)
+  int32_t S, C;                        // parts per row and cells per part (multiple of 32)
+  Partials part;                       // when S > 1
+  int* status;
+};
+
+int selected_pow2(int n_sel);
+cudaError_t launch_select_compact(const SelectedPlan& p, cudaStream_t stream);
+cudaError_t launch_selected(const SelectedPlan& p, cudaStream_t stream);
+
 // ---- combine (split_k_reduce) -------------------------------------------------
 // Folds the partial records of each (row, q head) in slot order with the sink.
 struct CombinePlan {
@@ -90,6 +116,7 @@ struct CombinePlan {
   const int32_t *row_begin, *row_end;    // slice scheme: n_used(r) from ranges ...
   int32_t N, C;
   const int32_t* n_used;                 // ... or from per-row counts (selected op)
+  const int32_t* row_len;                // ... or from per-row lengths with C (selected op)
   const int64_t* row_tiles;              // balanced scheme
   int32_t W;
   int use_pdl;

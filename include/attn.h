@@ -160,6 +160,8 @@ int32_t attn_prefill(const attn_args *args, void *ws, size_t ws_bytes, void *str
  * Each entry is a cudaEvent_t passed as void*, or NULL to skip it.          */
 int32_t attn_decode_timed(const attn_args *args, void *ws, size_t ws_bytes, void *stream,
                           void *const events[3]);
+int32_t attn_selected_timed(const attn_selected_args *args, void *ws, size_t ws_bytes, void *stream,
+                            void *const events[3]);
 
 /* attn_decode for callers that cannot allocate device memory (a real-time
  * loop that must not block in an allocator, a plugin with no memory pool of
