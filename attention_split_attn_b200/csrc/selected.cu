@@ -9,21 +9,23 @@
 // and empty rows as everywhere else (HartsyInference PR #910).
 //
 // B200 design:
-//  * select_compact_kernel: one CTA per row loads the list into shared memory,
-//    replaces entries outside [0, n_cells) by a sentinel, bitonic-sorts it and
-//    keeps each valid value once (flag + block scan).  The compacted list and
-//    its length go to the workspace (and to the caller's optional outputs).
-//  * selected_kernel: one CTA per (row, KV head, part).  A producer warp gathers
-//    each 32-cell block with one cp.async.bulk per K row and per V row (the
-//    cache row of a cell and head is D contiguous elements), completing on an
-//    mbarrier.  Rows land D*2+16 bytes apart so eight rows read at one column
-//    by ldmatrix fall in eight different bank groups.  The head dimension is
-//    split over D/64 consumer warps: warp w computes the partial scores of
-//    S^T = K Q^T over its 64 dimensions (m16n8k16, the q heads in N), the
-//    warps add their partials through shared memory in a fixed order, every
-//    warp then runs the same online softmax on the full scores, and warp w
-//    accumulates O^T += V^T P^T for its 64 dimensions.  Each consumer warp
-//    releases a stage as soon as it holds the block's fragments.
+//  * compaction, one CTA per row: for caches up to 256K cells a bitmap in
+//    shared memory (set a bit per valid entry, read the bits back in order
+//    with a popcount prefix scan); above that a bitonic sort of the list with
+//    invalid entries turned into a sentinel, keeping the first of each run.
+//    The compacted list and its length go to the workspace (and to the
+//    caller's optional outputs).
+//  * selected_kernel: one CTA per (row, KV head, part) with D/64 warps; warp w
+//    owns head dims [64w, 64w + 64).  Each warp gathers its column slice of
+//    every 32-cell block itself with 16-byte cp.async copies (rows past the
+//    list end zero-filled) into its own ring -- per-thread copies gather rows
+//    that mostly sit in L2 much faster than one bulk copy per row -- with rows
+//    144 bytes apart so ldmatrix reads are free of bank conflicts.  The warp
+//    computes the partial scores of S^T = K Q^T over its 64 dimensions
+//    (m16n8k16, the q heads in N), the warps add their partials through shared
+//    memory in a fixed order, every warp then runs the same online softmax on
+//    the full scores, and warp w accumulates O^T += V^T P^T for its dims.
+//    A warp refills a stage as soon as it holds the block's fragments.
 #include "common.cuh"
 #include "decode_tile.cuh"
 #include "internal.h"
@@ -37,6 +39,73 @@ constexpr int kSelTile = 32;   // cells per gathered block
 constexpr int kSortThreads = 1024;
 
 // ---- a2: sort + dedup of the selection lists ---------------------------------
+// For caches of at most kBitmapCells cells: one bit per cell in shared memory.
+// Setting the bit of every valid entry drops duplicates; reading the bits in
+// cell order (a popcount prefix over the words gives each bit its position)
+// yields the distinct valid entries in ascending order -- the same list the
+// sort-and-unique below produces, in O(n_sel + n_cells / 32).
+constexpr int kBitmapCells = 256 * 1024;
+
+__global__ void __launch_bounds__(kSortThreads) select_bitmap_kernel(const SelectedPlan p) {
+  extern __shared__ uint32_t bits[];          // [ceil(N / 32)] words, then [32] scan scratch
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int n = p.n_sel;
+  const int nw = (p.N + 31) / 32;
+  uint32_t* warp_tot = bits + nw;
+  for (int i = tid; i < nw; i += kSortThreads) bits[i] = 0u;
+  __syncthreads();
+  const int32_t* list = p.sel + (int64_t)r * p.sel_stride;
+  for (int i = tid; i < n; i += kSortThreads) {
+    const int32_t e = __ldg(list + i);
+    if (e >= 0 && e < p.N) atomicOr(&bits[e >> 5], 1u << (e & 31));
+  }
+  __syncthreads();
+  int32_t* out = p.compact + (int64_t)r * n;
+  int carry = 0;
+  for (int base = 0; base < nw; base += kSortThreads) {
+    const int i = base + tid;
+    uint32_t w = i < nw ? bits[i] : 0u;
+    const int cnt = __popc(w);
+    int x = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_tot[wid] = (uint32_t)x;
+    __syncthreads();
+    if (wid == 0) {
+      int t = (int)warp_tot[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, off);
+        if (lane >= off) t += y;
+      }
+      warp_tot[lane] = (uint32_t)t;
+    }
+    __syncthreads();
+    int pos = carry + x - cnt + (wid > 0 ? (int)warp_tot[wid - 1] : 0);
+    while (w) {
+      const int b = __ffs(w) - 1;
+      w &= w - 1;
+      const int32_t v = i * 32 + b;
+      out[pos] = v;
+      if (p.sorted_out) p.sorted_out[(int64_t)r * n + pos] = v;
+      ++pos;
+    }
+    carry += (int)warp_tot[31];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    p.count[r] = carry;
+    if (p.count_out) p.count_out[r] = carry;
+  }
+  if (p.sorted_out)
+    for (int i = carry + tid; i < n; i += kSortThreads) p.sorted_out[(int64_t)r * n + i] = -1;
+}
+
+// Larger caches: bitonic sort of the list in shared memory, then keep the
+// first of each run of equal valid values.
 __global__ void __launch_bounds__(kSortThreads) select_compact_kernel(const SelectedPlan p) {
   extern __shared__ int32_t sbuf[];           // [n_pow2] keys, then [kSortThreads/32] scan
   const int r = blockIdx.x, tid = threadIdx.x;
@@ -110,20 +179,35 @@ __global__ void __launch_bounds__(kSortThreads) select_compact_kernel(const Sele
 }
 
 // ---- the attention kernel --------------------------------------------------------
+// Warp w owns head dims [64w, 64w + 64) and gathers exactly that slice of each
+// 32-cell block's K and V rows itself: 16-byte cp.async copies (L2 only; per-
+// thread copies gather L2-resident rows far faster than one bulk copy per
+// row) into the warp's own ring, rows past the end of the list zero-filled.
+// The warps meet only to add their partial scores.
 template <typename KT, int D, int NH>
 struct SelCfg {
-  static constexpr int NW = D / 64;                   // consumer warps (64 dims each)
+  static constexpr int NW = D / 64;                   // warps (64 dims each)
   static constexpr int NT = NH / 8;                   // head n-tiles
-  static constexpr int RS = D * 2 + 16;               // shared-memory row stride (bytes)
-  static constexpr int TILE_BYTES = kSelTile * RS;    // K or V block
+  static constexpr int RS = 64 * 2 + 16;              // row stride of a warp's slice (bytes)
+  static constexpr int TILE_BYTES = kSelTile * RS;    // K or V slice of a block
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NS = D == 256 ? 2 : 3;         // ring stages
-  static constexpr int EXCH_FLOATS = NW * 32 * 8 * NT;   // partial S^T of every consumer warp
-  static constexpr int EXCH_OFF = NS * STAGE_BYTES;
-  static constexpr int BAR_OFF = EXCH_OFF + 2 * EXCH_FLOATS * 4;
-  static constexpr int TOTAL = BAR_OFF + 2 * NS * 8 + 16;
-  static constexpr int THREADS = 32 * (NW + 1);
+  static constexpr int NS = NW == 4 ? 2 : 3;          // ring stages per warp
+  static constexpr int RING_BYTES = NS * STAGE_BYTES;
+  static constexpr int EXCH_FLOATS = NW * 32 * 8 * NT;   // partial S^T of every warp
+  static constexpr int EXCH_OFF = NW * RING_BYTES;
+  static constexpr int TOTAL = EXCH_OFF + EXCH_FLOATS * 4;
+  static constexpr int THREADS = 32 * NW;
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 template <typename KT, int D, int NH>
 __global__ void __launch_bounds__(SelCfg<KT, D, NH>::THREADS)
@@ -132,9 +216,6 @@ selected_kernel(const SelectedPlan p) {
   using Op = MmaType<KT>;
   constexpr int NW = C::NW, NT = C::NT, NS = C::NS;
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* empty = full + NS;
-  int* abort_flag = reinterpret_cast<int*>(empty + NS);
   float* exch = reinterpret_cast<float*>(smem + C::EXCH_OFF);
 
   const int64_t bid = blockIdx.x;
@@ -144,63 +225,44 @@ selected_kernel(const SelectedPlan p) {
   const int count = __ldg(p.count + r);
   const int c_begin = min(count, part * p.C);
   const int c_end = (part == p.S - 1) ? count : min(count, c_begin + p.C);
-  if (p.S > 1 && c_begin >= c_end) {
-    pdl_launch_dependents();
-    return;
-  }
+  pdl_launch_dependents();
+  if (p.S > 1 && c_begin >= c_end) return;
   const int n_tiles = (c_end - c_begin + kSelTile - 1) / kSelTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], NW);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  pdl_launch_dependents();
   const int32_t* cells = p.compact + (int64_t)r * p.n_sel;
   const KT* kbase = static_cast<const KT*>(p.k);
   const KT* vbase = static_cast<const KT*>(p.v);
+  const int dw = warp * 64;
+  const uint32_t ring = smem_u32(smem + warp * C::RING_BYTES);
 
-  if (warp == NW) {
-    // ---------------- producer: gather 32-cell blocks ----------------
-    int issued = 0;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int st = t % NS;
-      if (t >= NS) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_bounded(&empty[st], ((t / NS) & 1) ^ 1, p.status);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          if (lane == 0) atomicExch(abort_flag, 1);
-          break;
-        }
+  // block t's cell of this lane's row (-1 past the end of the list)
+  auto block_cell = [&](int t) {
+    const int idx = c_begin + t * kSelTile + lane;
+    return (t < n_tiles && idx < c_end) ? __ldg(cells + idx) : -1;
+  };
+  // gather this warp's slice of block t into stage t % NS: lane l copies
+  // 16-byte chunk l % 8 of rows l / 8 + 4 i; one commit group per block
+  auto issue = [&](int t, int cl) {
+    if (t < n_tiles) {
+      const uint32_t st = ring + (t % NS) * C::STAGE_BYTES;
+      const int chunk = lane & 7;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = (lane >> 3) + 4 * i;
+        const int c = __shfl_sync(0xffffffffu, cl, row);
+        const bool valid = c >= 0;
+        const int64_t off = (int64_t)(valid ? c : 0) * p.kv_sc + (int64_t)g * p.kv_sh + dw + chunk * 8;
+        cp_async16(st + row * C::RS + chunk * 16, kbase + off, valid);
+        cp_async16(st + C::TILE_BYTES + row * C::RS + chunk * 16, vbase + off, valid);
       }
-      const int idx = c_begin + t * kSelTile + lane;
-      const bool valid = idx < c_end;
-      const int c = valid ? __ldg(cells + idx) : 0;
-      const unsigned m = __ballot_sync(0xffffffffu, valid);
-      unsigned char* sk = smem + st * C::STAGE_BYTES;
-      if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)__popc(m) * 2u * D * 2u);
-      __syncwarp();
-      if (valid) {
-        const int64_t off = (int64_t)c * p.kv_sc + (int64_t)g * p.kv_sh;
-        bulk_load(sk + lane * C::RS, kbase + off, D * 2, &full[st]);
-        bulk_load(sk + C::TILE_BYTES + lane * C::RS, vbase + off, D * 2, &full[st]);
-      }
-      issued = t + 1;
     }
-    if (lane == 0 && *(volatile int*)abort_flag)
-      for (int t = max(0, issued - NS); t < issued; ++t) mbar_wait_bounded(&full[t % NS], (t / NS) & 1, nullptr);
-    return;
-  }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int t = 0; t < NS; ++t) issue(t, block_cell(t));
 
-  // ---------------- consumers: warp w owns dims [64w, 64w + 64) ----------------
   const int grp = lane >> 2, tig = lane & 3;
   const int G = p.G, h0 = g * G;
-  const int dw = warp * 64;
   uint32_t qb[4][NT][2];
   {
     const KT* qrow = static_cast<const KT*>(p.q) + (int64_t)r * p.q_sr;
@@ -237,7 +299,7 @@ selected_kernel(const SelectedPlan p) {
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const int row = mt * 16 + (lane & 7) + (mi & 1) * 8;
-        const int chunk = (dw >> 3) + 2 * kk + (mi >> 1);
+        const int chunk = 2 * kk + (mi >> 1);
         koff[mt][kk] = row * C::RS + chunk * 16;
       }
 #pragma unroll
@@ -245,7 +307,7 @@ selected_kernel(const SelectedPlan p) {
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         const int row = ks * 16 + (lane & 7) + (mi >> 1) * 8;
-        const int chunk = (dw >> 3) + 2 * m4 + (mi & 1);
+        const int chunk = 2 * m4 + (mi & 1);
         voff[m4][ks] = C::TILE_BYTES + row * C::RS + chunk * 16;
       }
   }
@@ -258,20 +320,12 @@ selected_kernel(const SelectedPlan p) {
   float m[NT][2], l[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = neg_inf(), l[nt][0] = l[nt][1] = 0.f;
-  bool aborted = false;
-
   for (int t = 0; t < n_tiles; ++t) {
     const int st = t % NS;
-    // Every consumer warp takes part in the exchange barrier below, so after a
-    // timeout (here or in another warp) a warp stops waiting but keeps looping
-    // on whatever the stage holds; its output is poisoned at the end.
-    if (!aborted && *(volatile int*)abort_flag) aborted = true;
-    if (!aborted && !mbar_wait_bounded(&full[st], (t / NS) & 1, p.status)) {
-      atomicExch(abort_flag, 1);
-      aborted = true;
-    }
-    __syncwarp();
-    const uint32_t sbase = smem_u32(smem + st * C::STAGE_BYTES);
+    const int cl_next = block_cell(t + NS);   // indices of the block to gather next
+    cp_async_wait<NS - 1>();                  // this lane's copies of block t are done
+    __syncwarp();                             // ... and every other lane's
+    const uint32_t sbase = ring + st * C::STAGE_BYTES;
     uint32_t ka[2][4][4], va[4][2][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
@@ -283,8 +337,8 @@ selected_kernel(const SelectedPlan p) {
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks)
         ldsm_x4_trans(va[m4][ks][0], va[m4][ks][1], va[m4][ks][2], va[m4][ks][3], sbase + voff[m4][ks]);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
+    __syncwarp();                             // every lane holds block t: refill its stage
+    issue(t + NS, cl_next);
 
     // partial S^T over this warp's dims: [2 m-tiles of 16 cells][NT][4]
     float sc[2][NT][4];
@@ -299,23 +353,25 @@ selected_kernel(const SelectedPlan p) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) Op::mma(sc[mt][nt], ka[mt][kk], qb[kk][nt][0], qb[kk][nt][1]);
     if (NW > 1) {
-      // add the partials of all warps, in warp order
-      float* buf = exch + (t & 1) * C::EXCH_FLOATS;
-      float4* mine = reinterpret_cast<float4*>(buf + (warp * 32 + lane) * 8 * NT);
+      // add the partials of all warps, in warp order; layout [warp][fragment
+      // index][lane] so a warp's float4 stores and loads are contiguous
+      float4* buf = reinterpret_cast<float4*>(exch);
+      named_bar_sync(1, NW * 32);   // every warp has read the previous block's sums
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
-          mine[mt * NT + nt] = make_float4(sc[mt][nt][0], sc[mt][nt][1], sc[mt][nt][2], sc[mt][nt][3]);
+          buf[(warp * 2 * NT + mt * NT + nt) * 32 + lane] =
+              make_float4(sc[mt][nt][0], sc[mt][nt][1], sc[mt][nt][2], sc[mt][nt][3]);
       named_bar_sync(1, NW * 32);
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float4 s = reinterpret_cast<const float4*>(buf + lane * 8 * NT)[mt * NT + nt];
+          float4 s = buf[(mt * NT + nt) * 32 + lane];
 #pragma unroll
           for (int w = 1; w < NW; ++w) {
-            const float4 x = reinterpret_cast<const float4*>(buf + (w * 32 + lane) * 8 * NT)[mt * NT + nt];
+            const float4 x = buf[(w * 2 * NT + mt * NT + nt) * 32 + lane];
             s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
           }
           sc[mt][nt][0] = s.x; sc[mt][nt][1] = s.y; sc[mt][nt][2] = s.z; sc[mt][nt][3] = s.w;
@@ -425,7 +481,8 @@ selected_kernel(const SelectedPlan p) {
   }
 
   // ---------------- epilogue ----------------
-  aborted = aborted || (*(volatile int*)abort_flag != 0);
+  cp_async_wait<0>();                         // no copy is left in flight at exit
+  constexpr bool aborted = false;             // (no barrier waits in this kernel)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -501,6 +558,15 @@ int selected_pow2(int n_sel) {
 }
 
 cudaError_t launch_select_compact(const SelectedPlan& p, cudaStream_t stream) {
+  if (p.N <= kBitmapCells) {
+    // one bit per cell (at most 32 KB) + the scan scratch
+    const size_t smem = ((size_t)(p.N + 31) / 32 + 32) * sizeof(uint32_t);
+    static std::atomic<unsigned long long> smem_set{0ull};
+    cudaError_t e = set_smem_limit_once(smem_set, select_bitmap_kernel, (kBitmapCells / 32 + 32) * 4);
+    if (e != cudaSuccess) return e;
+    select_bitmap_kernel<<<dim3((unsigned)p.R), kSortThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  }
   // at most 4096 keys + the scan scratch: 16.5 KB, under the default limit
   const size_t smem = ((size_t)p.n_pow2 + kSortThreads / 32) * sizeof(int32_t);
   select_compact_kernel<<<dim3((unsigned)p.R), kSortThreads, smem, stream>>>(p);

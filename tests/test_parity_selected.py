@@ -158,3 +158,14 @@ def test_selected_prefill_workload_sampled(cuda_lib):
     rows = np.random.default_rng(3).choice(p.n_rows, size=48, replace=False)
     sub = p.row_subset(rows)
     check(sub, out[torch.from_numpy(rows).cuda()], "selected_prefill sample")
+
+
+def test_compaction_large_cache_sort_path(cuda_lib):
+    """Caches above 256K cells take the sort-and-unique compaction instead of
+    the bitmap one; both must give the oracle's list bit for bit."""
+    p = W.random_selected(26, R=3, Hq=4, Hkv=1, D=64, N=300000, n_sel=600, dup_frac=0.2)
+    out, srt, cnt = run_selected(p, want_compact=True)
+    ref_srt, ref_cnt = oracle.select_compact(p.sel, p.n_cells)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(srt.cpu().numpy(), ref_srt)
+    check(p, out, "large cache")
