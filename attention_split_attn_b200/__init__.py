@@ -31,7 +31,8 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
-           "attn_prefill", "attn_decode_timed", "attn_selected_timed", "attn_decode_noalloc",
+           "attn_prefill", "attn_decode_timed", "attn_selected_timed", "attn_prefill_timed",
+           "attn_decode_noalloc",
            "attn_check_device_status",
            "attn_strerror", "attn_last_error", "attn_abi_version")
 
@@ -95,9 +96,11 @@ def load_library():
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int32
                 fn.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
-            lib.attn_decode_timed.restype = ctypes.c_int32
-            lib.attn_decode_timed.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t,
-                                              ctypes.c_void_p, ctypes.c_void_p * 3]
+            for name in ("attn_decode_timed", "attn_prefill_timed"):
+                fn = getattr(lib, name)
+                fn.restype = ctypes.c_int32
+                fn.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t,
+                               ctypes.c_void_p, ctypes.c_void_p * 3]
             lib.attn_decode_noalloc.restype = ctypes.c_int32
             lib.attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
             lib.attn_selected.restype = ctypes.c_int32
@@ -224,6 +227,37 @@ def attn_decode_timed_args(args: AttnArgs, ws: Optional[torch.Tensor], events, s
 def decode(q, k, v, out, *, ws=None, stream=None, **kw):
     """Split-K decode attention into `out` (see include/attn.h)."""
     return attn_decode_args(make_args(q, k, v, out, **kw), ws=ws, stream=stream)
+
+
+def attn_prefill_args(args: AttnArgs, ws: Optional[torch.Tensor] = None, stream=None):
+    """attn_prefill on a prepared AttnArgs (workspace allocated if needed)."""
+    lib = load_library()
+    need = workspace_size(args, OP_PREFILL)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = _workspace(need, dev, ws)
+    st = lib.attn_prefill(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                          0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
+    _raise_if(st, "attn_prefill")
+    return ws
+
+
+def attn_prefill_timed_args(args: AttnArgs, ws: Optional[torch.Tensor], events, stream=None):
+    """attn_prefill that also records three torch.cuda.Events (before the tile
+    classifier, after the tensor-core kernel, after the last kernel)."""
+    lib = load_library()
+    handles = [None if e is None else e.cuda_event for e in events]
+    if any(h == 0 for h in handles):
+        raise ValueError("record each torch.cuda.Event once before passing it (torch creates it lazily)")
+    ev = (ctypes.c_void_p * 3)(*handles)
+    st = lib.attn_prefill_timed(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                                0 if ws is None else ws.numel() * ws.element_size(),
+                                _stream_handle(stream), ev)
+    _raise_if(st, "attn_prefill_timed")
+
+
+def prefill(q, k, v, out, *, ws=None, stream=None, **kw):
+    """Causal prefill attention into `out` (see include/attn.h)."""
+    return attn_prefill_args(make_args(q, k, v, out, **kw), ws=ws, stream=stream)
 
 
 def make_selected_args(q, k, v, out, sel, *, sorted_out=None, count_out=None, **kw):

@@ -324,6 +324,45 @@ SelWs selected_ws_layout(const attn_args* a, int n_sel, const SelShape& sh) {
   return w;
 }
 
+// ---- prefill planning ---------------------------------------------------------------
+constexpr int kPfTile = 128;   // rows and cells per prefill tile
+
+int32_t check_prefill(const attn_args* a) {
+  int32_t st = validate_common(a, ATTN_OP_PREFILL);
+  if (st != ATTN_OK) return st;
+  if (a->kv_type != ATTN_F16 && a->kv_type != ATTN_BF16)
+    return fail(ATTN_ERR_UNSUPPORTED, "prefill: K/V must be F16 or BF16");
+  if (a->q_type != a->kv_type) return fail(ATTN_ERR_UNSUPPORTED, "prefill: Q must be in the K/V dtype");
+  if (a->head_dim != 64 && a->head_dim != 128)
+    return fail(ATTN_ERR_UNSUPPORTED, "prefill: head_dim %d not in {64, 128}", a->head_dim);
+  if (a->n_rows > 0) {
+    if (!aligned16(a->q)) return fail(ATTN_ERR_UNSUPPORTED, "prefill: q must be 16-byte aligned");
+    if ((a->n_rows > 1 && (a->q_stride_row % 8)) || (a->n_head_q > 1 && (a->q_stride_head % 8)) ||
+        (a->n_rows > 1 && a->q_stride_row == 0) || (a->n_head_q > 1 && a->q_stride_head == 0))
+      return fail(ATTN_ERR_UNSUPPORTED, "prefill: q strides must be nonzero multiples of 16 bytes");
+  }
+  const int64_t n_rt = ((int64_t)a->n_rows + kPfTile - 1) / kPfTile;
+  const int G = a->n_head_q / a->n_head_kv;
+  const int64_t ctas = n_rt * a->n_head_kv * ((G + 1) / 2);
+  const int64_t n_kt = ((int64_t)a->n_cells + kPfTile - 1) / kPfTile;
+  if (ctas > 0x7fffffffLL || n_rt * n_kt + n_kt * a->n_head_kv > 0x7fffffffLL)
+    return fail(ATTN_ERR_UNSUPPORTED, "prefill: grid too large");
+  return ATTN_OK;
+}
+
+struct PrefillWs {
+  size_t vbad_off, total;
+};
+
+PrefillWs prefill_ws_layout(const attn_args* a) {
+  const size_t n_rt = ((size_t)a->n_rows + kPfTile - 1) / kPfTile;
+  const size_t n_kt = ((size_t)a->n_cells + kPfTile - 1) / kPfTile;
+  PrefillWs w;
+  w.vbad_off = align256(n_rt * n_kt);
+  w.total = w.vbad_off + align256(n_kt * a->n_head_kv);
+  return w;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -355,7 +394,8 @@ int32_t attn_supports(const attn_args* a, int32_t op) {
   switch (op) {
     case ATTN_OP_DECODE: return check_decode(a);
     case ATTN_OP_SELECTED: return check_selected_base(a);
-    default: return fail(ATTN_ERR_UNSUPPORTED, "op %d is not available in this build", op);
+    case ATTN_OP_PREFILL: return check_prefill(a);
+    default: return fail(ATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
 }
 
@@ -369,6 +409,7 @@ size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
     case ATTN_OP_SELECTED:
       if (n_sel < 1 || n_sel > kMaxSel) return 0;
       return selected_ws_layout(a, n_sel, plan_selected(a, n_sel, sms)).total;
+    case ATTN_OP_PREFILL: return prefill_ws_layout(a).total;
     default: return 0;
   }
 }
@@ -533,8 +574,75 @@ int32_t attn_selected_timed(const attn_selected_args* a, void* ws, size_t ws_byt
 }
 
 int32_t attn_prefill(const attn_args* a, void* ws, size_t ws_bytes, void* stream) {
-  (void)a; (void)ws; (void)ws_bytes; (void)stream;
-  return fail(ATTN_ERR_UNSUPPORTED, "attn_prefill is not available in this build");
+  return attn_prefill_timed(a, ws, ws_bytes, stream, nullptr);
+}
+
+int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* stream, void* const events[3]) {
+  int32_t st = check_prefill(a);
+  if (st != ATTN_OK) return st;
+  if (a->n_rows == 0) return ATTN_OK;
+  DeviceInfo* di = nullptr;
+  if ((st = device_info(&di)) != ATTN_OK) return st;
+  const PrefillWs wl = prefill_ws_layout(a);
+  if (wl.total > 0 && (ws == nullptr || ws_bytes < wl.total))
+    return fail(ATTN_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", wl.total, ws_bytes);
+  if (wl.total > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(ATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+
+  CUtensorMap tmQ, tmK, tmV;
+  memset(&tmQ, 0, sizeof(tmQ));
+  memset(&tmK, 0, sizeof(tmK));
+  memset(&tmV, 0, sizeof(tmV));
+  // Q as a [rows][heads][D] array with 128-row boxes; K and V with 128-cell boxes.
+  if ((st = make_kv_map(&tmQ, a->q, a->q_type, a->head_dim, a->n_head_q, a->n_rows, a->q_stride_row,
+                        a->q_stride_head, kPfTile, 64, true)) != ATTN_OK)
+    return st;
+  if (a->n_cells > 0) {
+    if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                          a->kv_stride_head, kPfTile, 64, true)) != ATTN_OK)
+      return st;
+    if ((st = make_kv_map(&tmV, a->v, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                          a->kv_stride_head, kPfTile, 64, true)) != ATTN_OK)
+      return st;
+  }
+
+  PrefillPlan p{};
+  p.R = a->n_rows; p.Hq = a->n_head_q; p.Hkv = a->n_head_kv; p.G = a->n_head_q / a->n_head_kv;
+  p.D = a->head_dim; p.N = a->n_cells; p.kv_type = a->kv_type;
+  p.v = a->v; p.kv_sc = a->kv_stride_cell; p.kv_sh = a->kv_stride_head;
+  p.out = OutSpec{a->out, a->out_type, a->o_stride_row, a->o_stride_head};
+  p.f = RowFilter{a->row_begin, a->row_end, a->cell_seq, a->row_seq, a->cell_pos, a->row_pos,
+                  a->causal, a->mask, a->mask_stride_row};
+  p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
+  p.n_rt = (a->n_rows + kPfTile - 1) / kPfTile;
+  p.n_kt = (a->n_cells + kPfTile - 1) / kPfTile;
+  p.n_pairs = (p.G + 1) / 2;
+  char* wsb = static_cast<char*>(ws);
+  p.cls = reinterpret_cast<uint8_t*>(wsb);
+  p.vbad = reinterpret_cast<uint8_t*>(wsb + wl.vbad_off);
+  // Softcap polynomial: x = u + u w (k3 + w (k5 + w k7)), w = u^2, the odd
+  // Taylor series of c tanh(u / c) through u^7, used for |u| <= c / 5.
+  if (a->softcap > 0.f) {
+    const double c = a->softcap, c2 = c * c;
+    p.cap_lim = (float)(0.2 * c);
+    p.k3 = (float)(-1.0 / (3.0 * c2));
+    p.k5 = (float)(2.0 / (15.0 * c2 * c2));
+    p.k7 = (float)(-17.0 / (315.0 * c2 * c2 * c2));
+  }
+  const int oes = dtype_size(a->out_type);
+  const int64_t ovec = 16 / oes;
+  p.out_vec = aligned16(a->out) && (a->n_rows <= 1 || a->o_stride_row % ovec == 0) &&
+              (a->n_head_q <= 1 || a->o_stride_head % ovec == 0);
+  p.mask_vec = a->mask && aligned16(a->mask) && (a->n_rows <= 1 || a->mask_stride_row % 4 == 0);
+  p.status = di->status;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  record_event(events, 0, s);
+  cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, s, nullptr);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+  record_event(events, 1, s);
+  record_event(events, 2, s);
+  return ATTN_OK;
 }
 
 int32_t attn_check_device_status(void* stream) {

@@ -105,6 +105,36 @@ int selected_pow2(int n_sel);
 cudaError_t launch_select_compact(const SelectedPlan& p, cudaStream_t stream);
 cudaError_t launch_selected(const SelectedPlan& p, cudaStream_t stream);
 
+// ---- causal prefill -----------------------------------------------------------
+// Tiles of 128 query rows x 128 cells.  A classifier kernel tags every (row
+// tile, cell tile) as skipped (no row sees any cell), full (every row sees
+// every cell and the mask adds exactly 0 there) or mixed, and every (cell
+// tile, KV head) whose V holds a non-finite value; the tensor-core kernel then
+// runs one CTA per (row tile, pair of q heads of one KV group).
+enum : uint8_t { kTileSkip = 0, kTileFull = 1, kTileMixed = 2, kTileMixedBadV = 3 };
+
+struct PrefillPlan {
+  int32_t R, Hq, Hkv, G, D, N;
+  int32_t kv_type;
+  const void* v;            // V cache (scanned for non-finite values)
+  int64_t kv_sc, kv_sh;     // its cell and head strides (elements)
+  OutSpec out;
+  RowFilter f;
+  Logits lg;
+  int32_t n_rt, n_kt;       // row tiles, cell tiles (128 each)
+  int32_t n_pairs;          // ceil(G / 2): CTAs per (row tile, KV head)
+  uint8_t* cls;             // workspace [n_rt][n_kt]
+  uint8_t* vbad;            // workspace [n_kt][Hkv]
+  float cap_lim;            // |scale * q.k| at or below which the softcap polynomial is used
+  float k3, k5, k7;         // softcap polynomial coefficients t_n / softcap^(n-1)
+  int32_t out_vec;          // output rows may be written with 16-byte stores
+  int32_t mask_vec;         // mask rows may be read with 16-byte loads
+  int* status;
+};
+
+cudaError_t launch_prefill(const PrefillPlan& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, cudaStream_t stream, cudaEvent_t after_classify);
+
 // ---- combine (split_k_reduce) -------------------------------------------------
 // Folds the partial records of each (row, q head) in slot order with the sink.
 struct CombinePlan {

@@ -1,0 +1,804 @@
+// prefill.cu -- causal prefill on the sm_100a tensor cores (tcgen05 + TMEM).
+//
+// Many query rows attend over the cache with the semantics of decode
+// (HartsyInference PR #910 "attention semantic correctness": softcap before
+// ALiBi, F32 mask bias added unnarrowed, per-head sinks, +0 for rows with no
+// visible cell, NaN propagated).  The two dense contractions, S = Q K^T and
+// O += P V, run as tcgen05.mma (kind::f16, f32 accumulators in tensor memory);
+// everything between them (logit transforms, visibility, online softmax) runs
+// on the CUDA cores of two softmax warpgroups.
+//
+// Two kernels:
+//  * prefill_classify_kernel tags each (128-row tile, 128-cell tile) as
+//    skipped / full / mixed from the visibility rules and the mask, and each
+//    (cell tile, KV head) whose V holds a non-finite value.  Skipped tiles are
+//    never loaded; full tiles need no per-element visibility or mask work;
+//    only mixed tiles read the mask.  (The split of masked work by tile class
+//    follows the pages' observation that masked cells cost time in dense
+//    paths: strix-llama.cpp PR #115 "Performance" discussion.)
+//  * prefill_kernel: one CTA per (row tile, two q heads of one KV group).  Both
+//    heads share every K and V tile, so each tile crosses L2 once per pair.
+//      warp 0       TMA producer: Q of both heads once, then K_j, V_j through
+//                   a 3-stage ring (128-byte swizzled boxes of 64 x 128).
+//      warp 1       allocates 512 TMEM columns and issues the MMAs:
+//                     S_i  (TMEM cols i*128 .. +128)  = Q_i K_j^T
+//                     O_i  (TMEM cols 256 + i*D ..)  += P_i V_j
+//                   S_i of tile j+1 is issued as soon as warpgroup i has
+//                   read S_i of tile j, so the tensor core computes the next
+//                   scores while the softmax of this tile runs.
+//      warps 2-5    softmax of head slot 0; warps 6-9: slot 1.  Thread t owns
+//                   query row t of the tile (TMEM lane t): it reads its row of
+//                   S with tcgen05.ld, applies the transforms, keeps the
+//                   running max m and sum l, writes P (16-bit) to shared
+//                   memory in the UMMA K-major 128-byte-swizzled layout, and
+//                   rescales its O row in TMEM only when the max grew by more
+//                   than ln 256 (lazy rescaling: the weights stay <= 256, and
+//                   m is the common reference of l and O, so the result is
+//                   the same softmax).
+//    Mixed tiles whose V has a non-finite value for this KV head take P V on
+//    the CUDA cores instead, over each row's visible cells only, so that a NaN
+//    in a cell a row cannot see never reaches that row through 0 * NaN.
+//  All mbarrier waits are bounded; a timeout records ATTN_ERR_DEVICE_TIMEOUT,
+//  raises a CTA-wide abort flag, drains copies in flight and frees TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tcgen05.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kPfRows = 128;   // query rows per tile (MMA M)
+constexpr int kPfCells = 128;  // cells per tile (MMA N of S, K of P V)
+
+// ---------------------------------------------------------------------------
+// tile classifier
+// ---------------------------------------------------------------------------
+
+struct RowVis {
+  int32_t rb, re, rs, rp;
+};
+
+__device__ __forceinline__ RowVis row_vis(const RowFilter& f, int r, int N) {
+  RowVis v;
+  v.rb = f.row_begin ? __ldg(f.row_begin + r) : 0;
+  v.re = f.row_end ? __ldg(f.row_end + r) : N;
+  v.rs = f.row_seq ? __ldg(f.row_seq + r) : 0;
+  v.rp = f.row_pos ? __ldg(f.row_pos + r) : v.re - v.rb - 1;
+  return v;
+}
+
+// Block (rt, kt) for blockIdx.x < n_rt * n_kt; block (kt, g) of the V scan
+// after that.  256 threads; thread t looks at cell t % 128 of the tile and
+// at rows t / 128, t / 128 + 2, ...
+__global__ void __launch_bounds__(256) prefill_classify_kernel(PrefillPlan p) {
+  pdl_launch_dependents();   // the prefill kernel may start its prologue
+  const int tid = threadIdx.x;
+  const int64_t b = blockIdx.x;
+  const int64_t n_cls = (int64_t)p.n_rt * p.n_kt;
+  if (b < n_cls) {
+    const int rt = (int)(b / p.n_kt), kt = (int)(b % p.n_kt);
+    const int c = kt * kPfCells + (tid & 127);
+    const bool cin = c < p.N;
+    const int32_t cs = (cin && p.f.cell_seq) ? __ldg(p.f.cell_seq + c) : 0;
+    const int32_t cpos_given = (cin && p.f.cell_pos) ? __ldg(p.f.cell_pos + c) : 0;
+    bool any = false, notfull = false;
+    const int r_end = min(p.R, (rt + 1) * kPfRows);
+    for (int r = rt * kPfRows + (tid >> 7); r < r_end; r += 2) {
+      const RowVis rv = row_vis(p.f, r, p.N);
+      bool vis = cin && c >= rv.rb && c < rv.re;
+      if (p.f.cell_seq) vis = vis && cs == rv.rs;
+      if (p.f.causal) {
+        const int32_t cp = p.f.cell_pos ? cpos_given : c - rv.rb;
+        vis = vis && cp <= rv.rp;
+      }
+      bool zero_bias = true;
+      if (p.f.mask && vis) {
+        const float mv = __ldg(p.f.mask + (int64_t)r * p.f.mask_sr + c);
+        vis = !(mv == neg_inf());
+        zero_bias = (mv == 0.f);
+      }
+      any |= vis;
+      notfull |= !(vis && zero_bias);
+    }
+    const int a = __syncthreads_or(any ? 1 : 0);
+    const int nf = __syncthreads_or(notfull ? 1 : 0);
+    if (tid == 0) p.cls[b] = !a ? kTileSkip : (nf ? kTileMixed : kTileFull);
+  } else {
+    const int64_t vb = b - n_cls;
+    const int kt = (int)(vb / p.Hkv), g = (int)(vb % p.Hkv);
+    // 16-byte chunks of the tile's V rows of head g: 128 cells x D/8 chunks.
+    // A 16-bit value is non-finite iff its exponent field is all ones.
+    const int per_row = p.D / 8;
+    const uint32_t e_lo = p.kv_type == ATTN_BF16 ? 0x7F80u : 0x7C00u;
+    bool bad = false;
+    for (int i = tid; i < kPfCells * per_row; i += 256) {
+      const int c = kt * kPfCells + i / per_row;
+      if (c >= p.N) continue;
+      const uint16_t* row = static_cast<const uint16_t*>(p.v) + (int64_t)c * p.kv_sc + (int64_t)g * p.kv_sh;
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + (i % per_row));
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        bad |= ((ws[k] & e_lo) == e_lo) | (((ws[k] >> 16) & e_lo) == e_lo);
+    }
+    const int any_bad = __syncthreads_or(bad ? 1 : 0);
+    if (tid == 0) p.vbad[(int64_t)kt * p.Hkv + g] = any_bad ? 1 : 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the tensor-core kernel: shared-memory layout and helpers
+// ---------------------------------------------------------------------------
+
+template <int D>
+struct PfLayout {
+  static constexpr int BOX = 128 * 128;                  // one TMA box: 128 rows x 128 B (64 values)
+  static constexpr int TILE = kPfRows * D * 2;           // a Q, K or V tile: D/64 boxes
+  static constexpr int PTILE = kPfRows * kPfCells * 2;   // a P tile: two boxes
+  static constexpr int NS = 3;                           // K/V ring stages (one tile each)
+  static constexpr int OFF_Q = 0;                        // [2 slots][TILE]
+  static constexpr int OFF_P = OFF_Q + 2 * TILE;         // [2 slots][PTILE]
+  static constexpr int OFF_KV = OFF_P + 2 * PTILE;       // [NS][TILE]
+  static constexpr int OFF_BAR = OFF_KV + NS * TILE;
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_done[2], mma_done
+  static constexpr int N_BAR = 1 + 2 * NS + 8 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;   // TMEM base address, abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
+  static constexpr int THREADS = 320;                    // 10 warps
+  static constexpr uint32_t TMEM_COLS = 512;             // S0, S1 (128 each), O0, O1 (D each)
+  static_assert(2 * 128 + 2 * D <= (int)TMEM_COLS, "TMEM columns");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ unsigned char* pf_align1024(unsigned char* p) {
+  const uint32_t a = smem_u32(p);
+  return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// Bounded wait that also gives up as soon as another thread of the CTA has
+// raised the abort flag.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        record_status(status, ATTN_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform form: every lane waits; the warp goes on only if all did.
+__device__ __forceinline__ bool pf_wait_warp(uint64_t* bar, uint32_t parity, int* status,
+                                             volatile int* abort_flag) {
+  const bool ok = pf_wait(bar, parity, status, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// S (TMEM, 128 x 128 f32) = Q (128 x D) . K (128 x D)^T; both operands K-major
+// 128-byte-swizzled boxes of 64 columns.  One MMA per 16 columns of D: inside a
+// box the start address advances by 32 bytes, across boxes by one box.
+template <int D>
+__device__ __forceinline__ void pf_issue_s(uint32_t d_tmem, uint32_t q_base, uint32_t k_base, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (uint32_t)(kk >> 2) * PfLayout<D>::BOX + (uint32_t)(kk & 3) * 32u;
+    umma_ss(d_tmem, umma_desc_sw128(q_base + off, 16, 1024), umma_desc_sw128(k_base + off, 16, 1024), idesc,
+            kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (TMEM, 128 x D f32) (+)= P (128 x 128, K-major) . V (128 cells x D, D
+// contiguous: MN-major).  V's 8-cell groups are 1024 bytes apart (SBO) and its
+// 64-column boxes one box apart (LBO); 16 cells per MMA.
+template <int D>
+__device__ __forceinline__ void pf_issue_pv(uint32_t d_tmem, uint32_t p_base, uint32_t v_base, uint32_t idesc,
+                                            bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kPfCells / 16; ++kk) {
+    const uint32_t a_off = (uint32_t)(kk >> 2) * PfLayout<D>::BOX + (uint32_t)(kk & 3) * 32u;
+    umma_ss(d_tmem, umma_desc_sw128(p_base + a_off, 16, 1024),
+            umma_desc_sw128(v_base + (uint32_t)kk * 2048u, PfLayout<D>::BOX, 1024), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Cell tiles of one row tile in order, skipping the empty ones.
+struct PfTiles {
+  const uint8_t* cls;    // this row tile's class row [n_kt]
+  const uint8_t* vbad;   // [n_kt][Hkv]
+  int n_kt, Hkv, g;
+  __device__ __forceinline__ int next(int kt) const {
+    while (kt < n_kt && cls[kt] == kTileSkip) ++kt;
+    return kt;
+  }
+  __device__ __forceinline__ int code(int kt) const {
+    int c = cls[kt];
+    if (c == kTileMixed && vbad[(int64_t)kt * Hkv + g]) c = kTileMixedBadV;
+    return c;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// softmax warpgroups
+// ---------------------------------------------------------------------------
+
+// Softcap x = c * tanh(u / c) of a raw logit u = scale * q.k.
+//  pf_cap_poly: the odd Taylor series of c tanh(u / c) through u^7,
+//    u + u w (k3 + w (k5 + w k7)) with w = u^2 and k_n = t_n / c^(n-1)
+//    (t_3 = -1/3, t_5 = 2/15, t_7 = -17/315); for |u| <= c/5 the truncation
+//    is below 2e-8 c.  No branch, FMA pipe only.
+//  pf_cap_exact: any u, tanh |y| = 1 - 2 / (e^{2|y|} + 1) with 2^x on the
+//    special-function unit; NaN stays NaN, +-inf gives +-c.
+__device__ __forceinline__ float pf_cap_poly(float u, float k3, float k5, float k7) {
+  const float w = u * u;
+  float h = fmaf(w, k7, k5);
+  h = fmaf(w, h, k3);
+  return fmaf(u * w, h, u);
+}
+__device__ __forceinline__ float pf_cap_exact(float u, float c) {
+  const float e = ex2((2.f * kLog2e) * (fabsf(u) / c));
+  const float t = 1.f - 2.f / (e + 1.f);
+  return copysignf(c * t, u);
+}
+__device__ __forceinline__ float pf_softcap(float u, const PrefillPlan& p) {
+  return fabsf(u) <= p.cap_lim ? pf_cap_poly(u, p.k3, p.k5, p.k7) : pf_cap_exact(u, p.lg.softcap);
+}
+
+__device__ __forceinline__ float pf_max8(const float* v) {
+  return fmax_nan(fmax_nan(fmax_nan(v[0], v[1]), fmax_nan(v[2], v[3])),
+                  fmax_nan(fmax_nan(v[4], v[5]), fmax_nan(v[6], v[7])));
+}
+
+// Logit transforms of one thread's row of a tile: x_i = softcap(scale s_i),
+// then + slope * -|row_pos - cell_pos| (AL 1: cell positions c - row_begin,
+// i.e. row_pos + row_begin - c0 - i = A - i; AL 2: explicit cell positions).
+// The feature set is a template so the unrolled loop holds no branch.  Also
+// returns the tile max (NaN-propagating, 8 independent partial maxima) and the
+// largest |scale s_i| (the softcap polynomial's range check).
+template <bool CAP, int AL>
+__device__ __forceinline__ void pf_transform(const uint32_t* raw, float* x, float scale, float k3, float k5,
+                                             float k7, float nslope, float A, float rpf, const int32_t* cpos,
+                                             float& mt, float& umax) {
+  float mx[8], ub[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = neg_inf(), ub[k] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPfCells; ++i) {
+    float u = __uint_as_float(raw[i]) * scale;
+    if (CAP) {
+      ub[i & 7] = fmaxf(ub[i & 7], fabsf(u));
+      u = pf_cap_poly(u, k3, k5, k7);
+    }
+    if (AL == 1) u = fmaf(nslope, fabsf(A - (float)i), u);
+    if (AL == 2) u = fmaf(nslope, fabsf(rpf - (float)__ldg(cpos + i)), u);
+    x[i] = u;
+    mx[i & 7] = fmax_nan(mx[i & 7], u);
+  }
+  mt = pf_max8(mx);
+  umax = fmaxf(fmaxf(fmaxf(ub[0], ub[1]), fmaxf(ub[2], ub[3])), fmaxf(fmaxf(ub[4], ub[5]), fmaxf(ub[6], ub[7])));
+}
+
+// The same with the exact softcap outside the polynomial's range (taken
+// only when some |scale s_i| of the warp's rows exceeds it).
+template <int AL>
+__device__ __forceinline__ void pf_transform_exact(const uint32_t* raw, float* x, const PrefillPlan& p, float nslope,
+                                                float A, float rpf, const int32_t* cpos, float& mt) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = neg_inf();
+#pragma unroll
+  for (int i = 0; i < kPfCells; ++i) {
+    float u = pf_softcap(__uint_as_float(raw[i]) * p.lg.scale, p);
+    if (AL == 1) u = fmaf(nslope, fabsf(A - (float)i), u);
+    if (AL == 2) u = fmaf(nslope, fabsf(rpf - (float)__ldg(cpos + i)), u);
+    x[i] = u;
+    mx[i & 7] = fmax_nan(mx[i & 7], u);
+  }
+  mt = pf_max8(mx);
+}
+
+// Mixed tiles: per-cell visibility (range, sequence, causal, mask != -inf)
+// and the mask bias; excluded cells become -inf and lose their bit in vis.
+// With explicit cell positions the ALiBi term is added here (the transform
+// skipped it: it may not read cell_pos past the cache end).
+__device__ __forceinline__ void pf_visibility(float* x, uint32_t* vis, const PrefillPlan& p, const RowVis& rv,
+                                           bool rvalid, int c0, const float* mrow, bool mask_vec, bool alibi_pos,
+                                           float nslope, float& mt) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = neg_inf();
+  const bool whole = c0 + kPfCells <= p.N;
+  float4 mv4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < kPfCells; ++i) {
+    const int c = c0 + i;
+    const bool cin = c < p.N;
+    bool vc = rvalid && cin && c >= rv.rb && c < rv.re;
+    if (p.f.cell_seq) vc = vc && cin && __ldg(p.f.cell_seq + c) == rv.rs;
+    int32_t cp = c - rv.rb;
+    if (p.f.cell_pos && cin) cp = __ldg(p.f.cell_pos + c);
+    if (p.f.causal) vc = vc && cp <= rv.rp;
+    float mv = 0.f;
+    if (mrow) {
+      if (mask_vec && whole) {
+        if ((i & 3) == 0) mv4 = __ldg(reinterpret_cast<const float4*>(mrow + c));
+        mv = (i & 3) == 0 ? mv4.x : (i & 3) == 1 ? mv4.y : (i & 3) == 2 ? mv4.z : mv4.w;
+      } else if (cin) {
+        mv = __ldg(mrow + c);
+      }
+      vc = vc && !(mv == neg_inf());
+    }
+    float u = x[i];
+    if (alibi_pos) u = fmaf(nslope, fabsf((float)(rv.rp - cp)), u);
+    u += mv;
+    u = vc ? u : neg_inf();
+    if (!vc) vis[i >> 5] &= ~(1u << (i & 31));
+    x[i] = u;
+    mx[i & 7] = fmax_nan(mx[i & 7], u);
+  }
+  mt = pf_max8(mx);
+}
+
+template <typename KT>
+__device__ __forceinline__ uint32_t pf_pack(float lo, float hi) {
+  if constexpr (Storage<KT>::kDtype == ATTN_BF16) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+  } else {
+    __half2 b = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+  }
+}
+
+template <typename KT>
+__device__ __forceinline__ float pf_widen(uint16_t bits) {
+  if constexpr (Storage<KT>::kDtype == ATTN_BF16) return __uint_as_float((uint32_t)bits << 16);
+  else return __half2float(__ushort_as_half(bits));
+}
+
+// 32 consecutive output values of one (row, head) starting at element `i0`.
+__device__ __forceinline__ void pf_store32(const OutSpec& o, int64_t i0, const float* v, bool vec) {
+  if (vec && o.type == ATTN_F32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(o.out) + i0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  } else if (vec) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(o.out) + i0);
+    const bool bf = o.type == ATTN_BF16;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = bf ? pf_pack<__nv_bfloat16>(v[8 * k + 2 * e], v[8 * k + 2 * e + 1])
+                  : pf_pack<__half>(v[8 * k + 2 * e], v[8 * k + 2 * e + 1]);
+      dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) store_from_float(o.out, i0 + e, o.type, v[e]);
+  }
+}
+
+template <typename KT, int D>
+__device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& tiles, unsigned char* sm,
+                                           uint64_t* bars, volatile int* abort_flag, uint32_t tmem, int rt,
+                                           int h, int slot, int quarter, int lane) {
+  const bool out_vec = p.out_vec != 0, mask_vec = p.mask_vec != 0;
+  using L = PfLayout<D>;
+  constexpr int NS = L::NS;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* s_full = bars + 1 + 2 * NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* pv_done = s_full + 6;
+  const int row_t = quarter * 32 + lane;
+  const int r = rt * kPfRows + row_t;
+  const bool rvalid = r < p.R;
+  const RowVis rv = rvalid ? row_vis(p.f, r, p.N) : RowVis{0, 0, 0, 0};
+  const bool alibi = p.lg.slopes != nullptr;
+  const float nslope = alibi ? -__ldg(p.lg.slopes + h) : 0.f;
+  const float scale = p.lg.scale;
+  const bool cap = p.lg.softcap > 0.f;
+  const int al = !alibi ? 0 : (p.f.cell_pos ? 2 : 1);   // ALiBi: off, affine, explicit cell positions
+  const float rpf = (float)rv.rp;
+  const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+  const uint32_t tS = lane_base + (uint32_t)slot * 128u;
+  const uint32_t tO = lane_base + 256u + (uint32_t)slot * D;
+  unsigned char* Ps = sm + L::OFF_P + slot * L::PTILE;
+  const float* mrow = (p.f.mask && rvalid) ? p.f.mask + (int64_t)r * p.f.mask_sr : nullptr;
+  constexpr float kLazy = 5.545177444479562f;   // ln 256: rescale only when the max grows by more
+
+  float m = neg_inf(), l = 0.f, mneg2 = 0.f;    // mneg2 = -m * log2(e) (0 while m = -inf)
+  int j = 0;
+  bool ok = true;
+  for (int kt = tiles.next(0); kt < tiles.n_kt; kt = tiles.next(kt + 1), ++j) {
+    const int code = tiles.code(kt);
+    if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t raw[kPfCells];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
+    tmem_wait_ld();
+
+    float x[kPfCells];
+    uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+    float mt, umax = 0.f;
+    const int c0 = kt * kPfCells;
+    const float A = (float)(rv.rp + rv.rb - c0);
+    const int32_t* cpos = p.f.cell_pos ? p.f.cell_pos + c0 : nullptr;
+    // full tiles: ALiBi in the transform; mixed tiles with explicit positions:
+    // in the visibility pass (cell_pos may end inside the tile)
+    const int al_t = (code == kTileFull || al == 1) ? al : 0;
+    switch ((cap ? 3 : 0) + al_t) {
+      case 0: pf_transform<false, 0>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+      case 1: pf_transform<false, 1>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+      case 2: pf_transform<false, 2>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+      case 3: pf_transform<true, 0>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+      case 4: pf_transform<true, 1>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+      default: pf_transform<true, 2>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+    }
+    if (cap && __any_sync(0xffffffffu, !(umax <= p.cap_lim))) {
+      // some logit outside the polynomial's range: redo the row from S
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
+      tmem_wait_ld();
+      if (al_t == 0) pf_transform_exact<0>(raw, x, p, nslope, A, rpf, cpos, mt);
+      else if (al_t == 1) pf_transform_exact<1>(raw, x, p, nslope, A, rpf, cpos, mt);
+      else pf_transform_exact<2>(raw, x, p, nslope, A, rpf, cpos, mt);
+    }
+    tc_fence_before();
+    mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
+    if (code != kTileFull) pf_visibility(x, vis, p, rv, rvalid, c0, mrow, mask_vec, al == 2, nslope, mt);
+
+    // lazy rescaling of the running state
+    const bool need = !(mt <= m + kLazy);   // NaN compares false: a NaN max always rescales
+    float factor = 1.f;
+    if (need) {
+      const float mn = fmax_nan(m, mt);
+      factor = ex2((m - mn) * kLog2e);        // 0 when m was -inf
+      l *= factor;
+      m = mn;
+      mneg2 = (m == neg_inf()) ? 0.f : -m * kLog2e;
+    }
+
+    // Weights, their sum, and P packed to 16 bits (64 registers instead of
+    // 128 while O is rescaled below).
+    float ls[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+    uint32_t pk[kPfCells / 2];
+#pragma unroll
+    for (int i = 0; i < kPfCells; i += 2) {
+      const float p0 = ex2(fmaf(x[i], kLog2e, mneg2));
+      const float p1 = ex2(fmaf(x[i + 1], kLog2e, mneg2));
+      ls[(i >> 1) & 7] += p0;
+      ls[(i >> 1) & 7] += p1;
+      pk[i / 2] = pf_pack<KT>(p0, p1);
+    }
+    l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+
+    // P V of the previous tile must be complete before its P buffer is
+    // overwritten and before O is rescaled.
+    if (j > 0) {
+      if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p.status, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+    }
+    if (j > 0 && code != kTileMixedBadV && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tO + ch * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+        tmem_st32(tO + ch * 32, o);
+      }
+      tmem_wait_st();
+    }
+
+    // P row in the K-major 128-byte-swizzled layout the MMA reads: cells
+    // 0-63 in the first box, 64-127 in the second; 16-byte chunk k of row t
+    // at chunk k ^ (t & 7).
+#pragma unroll
+    for (int k8 = 0; k8 < kPfCells / 8; ++k8) {
+      const uint4 w = make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
+      const uint32_t off = (uint32_t)(k8 >> 3) * L::BOX + (uint32_t)row_t * 128u +
+                           ((uint32_t)((k8 & 7) ^ (row_t & 7)) << 4);
+      *reinterpret_cast<uint4*>(Ps + off) = w;
+    }
+
+    if (code == kTileMixedBadV) {
+      // P V on the CUDA cores over this row's visible cells only.
+      const int64_t LV = 2 * (int64_t)j + 1;
+      const int stV = (int)(LV % NS);
+      if (!pf_wait_warp(&kv_full[stV], (uint32_t)((LV / NS) & 1), p.status, abort_flag)) { ok = false; break; }
+      const unsigned char* Vs = sm + L::OFF_KV + stV * L::TILE;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float o[32];
+        uint32_t ou[32];
+        if (j > 0) {
+          tmem_ld32(tO + ch * 32, ou);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(ou[e]) * factor;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+#pragma unroll 2
+        for (int c = 0; c < kPfCells; ++c) {
+          const uint32_t vw = c < 64 ? (c < 32 ? vis[0] : vis[1]) : (c < 96 ? vis[2] : vis[3]);
+          if (!((vw >> (c & 31)) & 1u)) continue;
+          const uint32_t poff = (uint32_t)(c >> 6) * L::BOX + (uint32_t)row_t * 128u +
+                                ((uint32_t)(((c & 63) >> 3) ^ (row_t & 7)) << 4) + (uint32_t)(c & 7) * 2u;
+          const float pc = pf_widen<KT>(*reinterpret_cast<const uint16_t*>(Ps + poff));
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const int d = ch * 32 + q8 * 8;
+            const uint32_t voff = (uint32_t)(d >> 6) * L::BOX + (uint32_t)c * 128u +
+                                  ((uint32_t)(((d & 63) >> 3) ^ (c & 7)) << 4);
+            float vf[8];
+            unpack_vec<KT>(*reinterpret_cast<const uint4*>(Vs + voff), vf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[q8 * 8 + e] = fmaf(pc, vf[e], o[q8 * 8 + e]);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e]);
+        tmem_st32(tO + ch * 32, ou);
+      }
+      tmem_wait_st();
+    } else {
+      fence_async_smem();   // P visible to the tensor core
+    }
+    tc_fence_before();
+    mbar_arrive(&p_full[slot]);
+  }
+
+  if (!ok) return;
+  if (j > 0) {
+    if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p.status, abort_flag)) return;
+    tc_fence_after();
+  }
+  // Fold with the sink (an extra logit with no value vector) and normalise.
+  const float sigma = p.lg.sinks ? __ldg(p.lg.sinks + h) : neg_inf();
+  const float Mf = fmax_nan(m, sigma);
+  const bool is_nan = isnan(Mf), is_zero = (Mf == neg_inf());
+  float f = 0.f;
+  if (!is_nan && !is_zero) {
+    const float fo = ex2((m - Mf) * kLog2e);
+    const float Lf = l * fo + ex2((sigma - Mf) * kLog2e);
+    f = fo / Lf;
+  }
+  const int64_t ob = rvalid ? (int64_t)r * p.out.sr + (int64_t)h * p.out.sh : 0;
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t ou[32];
+    if (j > 0) {
+      tmem_ld32(tO + ch * 32, ou);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ou[e] = 0u;
+    }
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = is_nan ? qnan() : (is_zero ? 0.f : __uint_as_float(ou[e]) * f);
+    if (rvalid) pf_store32(p.out, ob + ch * 32, v, out_vec);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+
+// One CTA per (row tile, KV head g, pair of q heads of g).  Heavier row tiles
+// (later rows see more cells under causality) are launched first.
+template <typename KT, int D>
+__global__ void __launch_bounds__(PfLayout<D>::THREADS, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const PrefillPlan p) {
+  using L = PfLayout<D>;
+  constexpr int NS = L::NS;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = pf_align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + NS;
+  uint64_t* s_full = bars + 1 + 2 * NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* pv_done = s_full + 6;
+  uint64_t* mma_done = s_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_rt = p.Hkv * p.n_pairs;
+  const int rt = p.n_rt - 1 - (int)(blockIdx.x / per_rt);
+  const int g = (int)(blockIdx.x % per_rt) / p.n_pairs;
+  const int pair = (int)(blockIdx.x % per_rt) % p.n_pairs;
+  const int h0 = g * p.G + 2 * pair;
+  const bool two = 2 * pair + 1 < p.G;
+  const int n_slots = two ? 2 : 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], kPfRows);
+      mbar_init(&p_full[s], kPfRows);
+      mbar_init(&pv_done[s], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, L::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait_prior_grid();   // tile classes from the classifier
+
+  const PfTiles tiles{p.cls + (int64_t)rt * p.n_kt, p.vbad, p.n_kt, p.Hkv, g};
+
+  if (warp == 0) {
+    // ---- TMA producer ----
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int kt = tiles.next(0);
+      int64_t Lc = 0;   // loads issued into the ring
+      bool ok = true;
+      const bool any = kt < p.n_kt;
+      if (any) {
+        mbar_arrive_expect_tx(q_full, (uint32_t)(n_slots * L::TILE));
+        for (int s = 0; s < n_slots; ++s)
+#pragma unroll
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, q_full, bx * 64, h0 + s, rt * kPfRows,
+                        pol);
+      }
+      for (; ok && kt < p.n_kt; kt = tiles.next(kt + 1)) {
+        for (int kv = 0; kv < 2; ++kv) {
+          const int st = (int)(Lc % NS);
+          if (Lc >= NS && !pf_wait(&kv_empty[st], (uint32_t)(((Lc / NS) + 1) & 1), p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[st], (uint32_t)L::TILE);
+#pragma unroll
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_3d(sm + L::OFF_KV + st * L::TILE + bx * L::BOX, kv ? &tmV : &tmK, &kv_full[st], bx * 64, g,
+                        kt * kPfCells, pol);
+          ++Lc;
+        }
+      }
+      // leave no copy in flight (bounded; completed loads return at once)
+      for (int64_t k = Lc > NS ? Lc - NS : 0; k < Lc; ++k)
+        mbar_wait_bounded(&kv_full[k % NS], (uint32_t)((k / NS) & 1), nullptr);
+      if (any) mbar_wait_bounded(q_full, 0, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr int bf = Storage<KT>::kDtype == ATTN_BF16 ? 1 : 0;
+      constexpr uint32_t idS = umma_idesc_f16(kPfRows, kPfCells, bf, 0, 0);
+      constexpr uint32_t idO = umma_idesc_f16(kPfRows, D, bf, 0, 1);
+      const uint32_t q_addr = smem_u32(sm + L::OFF_Q), p_addr = smem_u32(sm + L::OFF_P);
+      const uint32_t kv_addr = smem_u32(sm + L::OFF_KV);
+      int kt = tiles.next(0);
+      bool ok = kt < p.n_kt;
+      if (ok) {
+        ok = pf_wait(q_full, 0, p.status, abort_flag) && pf_wait(&kv_full[0], 0, p.status, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          for (int s = 0; s < n_slots; ++s) {
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr, idS);
+            umma_commit(&s_full[s]);
+          }
+          umma_commit(&kv_empty[0]);
+        }
+      }
+      for (int64_t j = 0; ok && kt < p.n_kt; ++j) {
+        const int kn = tiles.next(kt + 1);
+        const bool has_next = kn < p.n_kt;
+        const bool pv_mma = tiles.code(kt) != kTileMixedBadV;
+        const int64_t LK = 2 * (j + 1), LV = 2 * j + 1;
+        const int stK = (int)(LK % NS), stV = (int)(LV % NS);
+        if (has_next && !pf_wait(&kv_full[stK], (uint32_t)((LK / NS) & 1), p.status, abort_flag)) break;
+        if (!pf_wait(&kv_full[stV], (uint32_t)((LV / NS) & 1), p.status, abort_flag)) break;
+        tc_fence_after();
+        for (int s = 0; s < n_slots && ok; ++s) {
+          if (has_next) {
+            if (!pf_wait(&s_free[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr + stK * L::TILE, idS);
+            umma_commit(&s_full[s]);
+            if (s == n_slots - 1) umma_commit(&kv_empty[stK]);
+          }
+          if (!pf_wait(&p_full[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          if (pv_mma)
+            pf_issue_pv<D>(tmem + 256u + (uint32_t)s * D, p_addr + s * L::PTILE, kv_addr + stV * L::TILE, idO,
+                           j > 0);
+          umma_commit(&pv_done[s]);
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[stV]);
+        kt = kn;
+      }
+      umma_commit(mma_done);   // arrives once every MMA issued above has retired
+    }
+  } else {
+    // ---- softmax warpgroups ----
+    const int slot = (warp - 2) >> 2;
+    if (slot < n_slots)
+      pf_softmax<KT, D>(p, tiles, sm, bars, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    mbar_wait_bounded(mma_done, 0, p.status);
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+template <typename KT, int D>
+cudaError_t launch_prefill_t(const PrefillPlan& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, cudaStream_t stream, cudaEvent_t after_classify) {
+  using L = PfLayout<D>;
+  auto kern = prefill_kernel<KT, D>;
+  static std::atomic<unsigned long long> smem_set{0ull};
+  cudaError_t e = set_smem_limit_once(smem_set, kern, L::SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t n_cls = (int64_t)p.n_rt * p.n_kt, n_scan = (int64_t)p.n_kt * p.Hkv;
+  if (n_cls + n_scan > 0) {
+    prefill_classify_kernel<<<(unsigned)(n_cls + n_scan), 256, 0, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (after_classify) cudaEventRecord(after_classify, stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((int64_t)p.n_rt * p.Hkv * p.n_pairs));
+  cfg.blockDim = dim3(L::THREADS);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = after_classify ? 0 : 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmQ, tmK, tmV, p);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillPlan& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, cudaStream_t stream, cudaEvent_t after_classify) {
+  const bool bf = p.kv_type == ATTN_BF16;
+  if (p.D == 64)
+    return bf ? launch_prefill_t<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, stream, after_classify)
+              : launch_prefill_t<__half, 64>(p, tmQ, tmK, tmV, stream, after_classify);
+  return bf ? launch_prefill_t<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, stream, after_classify)
+            : launch_prefill_t<__half, 128>(p, tmQ, tmK, tmV, stream, after_classify);
+}
+
+}  // namespace attn

@@ -305,6 +305,54 @@ def random_problem(seed: int, R: int = 3, Hq: int = 4, Hkv: int = 2, D: int = 64
     return p
 
 
+def random_prefill(seed: int, R: int = 130, Hq: int = 4, Hkv: int = 2, D: int = 128,
+                   depth: int = 300, kv_dtype=BF16, out_dtype=F32, causal_by: str = "flag",
+                   softcap: float = 0.0, alibi: bool = False, sinks: bool = False,
+                   bias_frac: float = 0.0, nan_v: int = 0, extra_cells: int = 0,
+                   value_scale: float = 1.0, scale: Optional[float] = None) -> Problem:
+    """R new query rows at positions depth .. depth+R-1 over a cache of
+    depth + R cells (plus `extra_cells` later cells no row may see).
+    causal_by: "flag" (causal flag, row positions, affine cell positions),
+    "pos" (causal flag with explicit cell positions), "mask" (an F32 mask of
+    0 / -inf carries causality, causal flag off).  bias_frac: that fraction of
+    mask entries on visible cells get a finite N(0,1) bias (mask mode only).
+    nan_v: that many cells of the last R (each visible to some rows only) get a
+    NaN in one V element of every KV head."""
+    rng = np.random.default_rng(seed)
+    N = depth + R + extra_cells
+    q = (_normal(rng, (R, Hq, D), F32) * value_scale).to(kv_dtype)
+    k = (_normal(rng, (N, Hkv, D), F32) * value_scale).to(kv_dtype)
+    v = _normal(rng, (N, Hkv, D), kv_dtype)
+    rpos = depth + np.arange(R, dtype=np.int64)
+    p = Problem("random_prefill", q, k, v, out_dtype=out_dtype,
+                scale=(1.0 / math.sqrt(D)) if scale is None else scale, softcap=softcap,
+                row_pos=_i32(rpos))
+    if causal_by in ("flag", "pos"):
+        p.causal = True
+        if causal_by == "pos":
+            p.cell_pos = _i32(np.arange(N))
+    elif causal_by == "mask":
+        cols = np.arange(N, dtype=np.int64)
+        m = np.where(cols[None, :] <= rpos[:, None], np.float32(0.0), np.float32(-np.inf))
+        if bias_frac > 0:
+            hit = (rng.random((R, N)) < bias_frac) & (m == 0)
+            m[hit] = rng.standard_normal(int(hit.sum())).astype(np.float32)
+        p.mask = torch.from_numpy(m)
+    else:
+        raise ValueError(causal_by)
+    if nan_v:
+        cells = rng.choice(np.arange(depth, depth + R), size=min(nan_v, R), replace=False)
+        vv = p.v.clone()
+        for c in cells:
+            vv[int(c), :, int(rng.integers(D))] = float("nan")
+        p.v = vv
+    if alibi:
+        p.alibi_slopes = alibi_slopes_textbook(Hq)
+    if sinks:
+        p.sinks = torch.from_numpy(rng.standard_normal(Hq).astype(np.float32))
+    return p
+
+
 def random_selected(seed: int, R: int = 4, Hq: int = 8, Hkv: int = 2, D: int = 64,
                     N: int = 200, n_sel: int = 96, kv_dtype=F16, out_dtype=F32,
                     inv_frac: float = 0.05, dup_frac: float = 0.1, softcap: float = 0.0,

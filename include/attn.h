@@ -19,8 +19,16 @@
  *                  the GPU.  Defined by strix-llama.cpp PR #115 / #119
  *                  (FLASH_ATTN_EXT with a selection list src[5];
  *                  flash_attn_sel.comp; flash_attn_split_k_reduce).
- *   attn_prefill   causal prefill: many query rows over the cache, QK^T and PV
- *                  on the tensor cores, same semantics as decode.
+ *   attn_prefill   causal prefill: many query rows over the cache with the
+ *                  semantics below (softcap before ALiBi, F32 mask bias,
+ *                  sinks, +0 for excluded rows, NaN propagation; HartsyInference
+ *                  PR #910).  QK^T and PV run on the tensor cores in tiles of
+ *                  128 rows x 128 cells; P is rounded to the K/V dtype before
+ *                  PV.  Supported: K/V and Q in F16 or BF16 (same dtype),
+ *                  head_dim 64 or 128, Q 16-byte aligned with strides that are
+ *                  multiples of 16 bytes; any out dtype.  n_slices, max_row_len
+ *                  and grid_order are ignored.  Workspace: one byte per
+ *                  (128-row tile, 128-cell tile) and per (cell tile, KV head).
  *
  * Semantics (all three; HartsyInference PR #910 "attention semantic
  * correctness"):  for row r and query head h (KV head g = h / (Hq/Hkv)),
@@ -162,6 +170,8 @@ int32_t attn_decode_timed(const attn_args *args, void *ws, size_t ws_bytes, void
                           void *const events[3]);
 int32_t attn_selected_timed(const attn_selected_args *args, void *ws, size_t ws_bytes, void *stream,
                             void *const events[3]);
+int32_t attn_prefill_timed(const attn_args *args, void *ws, size_t ws_bytes, void *stream,
+                           void *const events[3]);
 
 /* attn_decode for callers that cannot allocate device memory (a real-time
  * loop that must not block in an allocator, a plugin with no memory pool of
