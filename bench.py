@@ -15,6 +15,15 @@ synchronize, timed with CUDA events on the launching stream, max over ranks.
 Each step reads a different one of three resident input sets (~0.9 GB of K/V
 in all), so a step never finds the previous step's cache in L2 (126 MB).
 
+The line's "parts" object times the other two operations on their own
+workloads, per call with the L2 flushed before each call: maskless
+selected-key attention (2048 rows, GQA 12, D 256, fp16 cache of 32768 cells;
+effective GB/s of the gathered K/V rows) and causal prefill (2048 rows over
+14048 cells, Hq 64 / Hkv 8, D 128, bf16; TFLOP/s over the visible pairs on
+the tensor cores), each with the roofline of its main kernel.
+--profile-op {decode,selected,prefill} only runs W + K calls of one operation
+(the command the ncu summaries under profiles/ are taken on).
+
 --impl reference times the FP64 CPU oracle on the host cores on a bounded
 sample of the same workload (the pages ship no code; the oracle is the
 baseline arm).  Under torchrun every rank runs its own batch (weak scaling;
@@ -255,9 +264,10 @@ def run_ours(args, rank, world, local):
     main_ms = [e[0].elapsed_time(e[1]) for e in ev]
     kmean_ms = sum(main_ms) / len(main_ms)
     achieved = step_bytes / (kmean_ms * 1e-3) / 1e9
-    traffic = _recorded_traffic()
+    traffic = _recorded_traffic("decode_stream_kernel")
 
     e2e = run_e2e(args, sets, stream)
+    parts = None if args.no_parts else run_parts(args, rank, dev, stream)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
@@ -275,24 +285,168 @@ def run_ours(args, rank, world, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if parts is not None:
+        line["parts"] = parts
+        line["gpu_launches"] += sum(p_["gpu_launches"] for p_ in parts.values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def _recorded_traffic():
-    """DRAM bytes per launch of the slice kernel from the committed ncu summary,
-    if it was taken on the current kernel build (else null)."""
-    path = os.path.join(ROOT, "profiles", "decode_slice_kernel_gqa_decode.json")
+def _recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/traffic.json), if it was taken on the current sources (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f)
-    src = os.path.join(ROOT, "attention_split_attn_b200", "csrc", "decode.cu")
-    import hashlib
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return d.get("dram_bytes_per_launch") if d.get("decode_cu_sha256_16") == h else None
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    m = hashlib.sha256()
+    for name in d["sources"]:
+        with open(os.path.join(ROOT, "attention_split_attn_b200", "csrc", name), "rb") as f:
+            m.update(f.read())
+    return d["dram_bytes_per_launch"] if m.hexdigest()[:16] == d["sources_sha256_16"] else None
+
+
+class _L2Flush:
+    """Writes a 256 MiB buffer (twice the L2) between timed calls."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def _time_calls(call_timed, n, flush, stream):
+    """n calls, each bracketed by its own events on the launching stream with
+    an L2 flush before it; returns (mean whole-call ms, mean main-kernel ms)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush()
+        call_timed(ev[i])
+    torch.cuda.synchronize()
+    whole = [e[0].elapsed_time(e[2]) for e in ev]
+    main = [e[0].elapsed_time(e[1]) for e in ev]
+    return sum(whole) / n, sum(main) / n
+
+
+def selected_bytes(p) -> int:
+    """K and V rows of every distinct valid selected cell for each KV head,
+    plus Q, the selection lists and the output."""
+    sel = p.sel.numpy()
+    n_valid = 0
+    for row in sel:
+        v = row[(row >= 0) & (row < p.n_cells)]
+        n_valid += len(np.unique(v))
+    kv = n_valid * p.n_head_kv * p.head_dim * p.k.element_size() * 2
+    o = p.n_rows * p.n_head_q * p.head_dim * torch.empty((), dtype=p.out_dtype).element_size()
+    return kv + p.q.numel() * p.q.element_size() + sel.size * 4 + o
+
+
+def prefill_flops(p) -> int:
+    """4 D flops (QK^T and PV) per visible (row, cell, q head); visibility is
+    carried by the mask in the causal prefill workload."""
+    vis = int(torch.isfinite(p.mask).sum()) if p.mask is not None else p.n_rows * p.n_cells
+    return 4 * p.head_dim * vis * p.n_head_q
+
+
+def run_parts(args, rank, dev, stream):
+    """The selected-key and causal-prefill workloads, each timed per call
+    (L2 flushed before every call), with the roofline of its main kernel."""
+    hbm_peak, tc_peak, peak_kind = _peaks()
+    flush = _L2Flush(dev)
+    n = max(3, min(args.steps, 20))
+    parts = {}
+
+    # maskless selected-key: 2048 rows, GQA 12, D 256, fp16 cache of 32768 cells
+    p = W.selected_prefill()
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    sel = kw.pop("sel")
+    sa = A.make_selected_args(q, k, v, out, sel, **kw)
+    ws = torch.empty(max(A.selected_workspace_size(sa), 256), dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        A.attn_selected_args(sa, ws=ws, stream=stream)
+    whole, main = _time_calls(lambda e: A.attn_selected_timed_args(sa, ws, e, stream=stream), n, flush, stream)
+    nbytes = selected_bytes(p)
+    parts["selected"] = {
+        "workload": "selected_prefill: 2048 rows, Hq 48 / Hkv 4, D 256, fp16 KV of 32768 cells, "
+                    "2048-entry lists (5% dup, 3% invalid), f32 out",
+        "value": nbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (effective: gathered K/V bytes)",
+        "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
+        "gpu_launches": 3 * n,
+        "roofline": {"bound": "hbm", "achieved": nbytes / (main * 1e-3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak,
+                     "traffic": _recorded_traffic("selected_kernel"),
+                     "kernel": "select_bitmap_kernel + selected_kernel",
+                     "kernel_ms": main, "algorithmic_bytes": nbytes,
+                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy); gathered rows are mostly L2 hits"},
+    }
+    del q, k, v, out, sel, sa, ws, kw
+
+    # causal prefill: 2048 rows over 14048 cells, Hq 64 / Hkv 8, D 128, bf16
+    p = W.causal_prefill()
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    pa = A.make_args(q, k, v, out, **kw)
+    ws = torch.empty(max(A.workspace_size(pa, A.OP_PREFILL), 256), dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        A.attn_prefill_args(pa, ws=ws, stream=stream)
+    whole, main = _time_calls(lambda e: A.attn_prefill_timed_args(pa, ws, e, stream=stream), n, flush, stream)
+    flops = prefill_flops(p)
+    parts["prefill"] = {
+        "workload": "causal_prefill: 2048 rows over 14048 cells (depth 12000), Hq 64 / Hkv 8, D 128, "
+                    "bf16, softcap 50, ALiBi, sinks, f32 causal mask",
+        "value": flops / (whole * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
+        "gpu_launches": 2 * n,
+        "roofline": {"bound": "tensor", "achieved": flops / (main * 1e-3) / 1e12, "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": flops / (main * 1e-3) / 1e12 / tc_peak,
+                     "traffic": _recorded_traffic("prefill_kernel"),
+                     "kernel": "prefill_classify_kernel + prefill_kernel (tcgen05)",
+                     "kernel_ms": main, "algorithmic_flops": flops,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS)"},
+    }
+    return parts
+
+
+def run_profile_op(args, local):
+    """--profile-op: W + K plain calls of one operation on its benchmark
+    workload and nothing else (the command the ncu summaries are taken on)."""
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    A.load_library()
+    op = args.profile_op
+    if op == "decode":
+        p = W.gqa_decode(poison_unused=False)
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_decode_args(a, ws=ws)
+    elif op == "selected":
+        p = W.selected_prefill()
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        sel = kw.pop("sel")
+        a = A.make_selected_args(q, k, v, out, sel, **kw)
+        ws = torch.empty(max(A.selected_workspace_size(a), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_selected_args(a, ws=ws)
+    else:
+        p = W.causal_prefill()
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_PREFILL), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_prefill_args(a, ws=ws)
+    for _ in range(args.warmup + args.steps):
+        call()
+    torch.cuda.synchronize()
+    A.check_device_status()
+    print(json.dumps({"profile_op": op, "calls": args.warmup + args.steps}), flush=True)
 
 
 def run_e2e(args, sets, stream):
@@ -344,11 +498,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-parts", action="store_true", help="time the decode workload only")
+    ap.add_argument("--profile-op", choices=["decode", "selected", "prefill"], default=None,
+                    help="only run W + K calls of one operation (for ncu captures); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     rank, world, local = _dist()
     try:
-        if args.impl == "reference":
+        if args.profile_op:
+            run_profile_op(args, local)
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local)
