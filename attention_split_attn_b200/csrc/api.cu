@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -628,6 +629,16 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
     p.k3 = (float)(-1.0 / (3.0 * c2));
     p.k5 = (float)(2.0 / (15.0 * c2 * c2));
     p.k7 = (float)(-17.0 / (315.0 * c2 * c2 * c2));
+    const double sc = a->scale, s2 = sc * sc;
+    const double a3 = p.k3 * sc * s2, a5 = p.k5 * sc * s2 * s2, a7 = p.k7 * sc * s2 * s2 * s2;
+    auto normal = [](double v) { return std::fabs(v) >= 1.1754943508222875e-38 && std::fabs(v) <= 3.0e38; };
+    if (sc != 0.0 && std::isfinite(sc) && normal(a3) && normal(a5) && normal(a7) && normal(0.2 * c / std::fabs(sc))) {
+      p.a3 = (float)a3;
+      p.a5 = (float)a5;
+      p.a7 = (float)a7;
+      p.s_lim = (float)(0.2 * c / std::fabs(sc));
+      p.cap_raw = 1;
+    }
   }
   const int oes = dtype_size(a->out_type);
   const int64_t ovec = 16 / oes;

@@ -127,6 +127,12 @@ struct PrefillPlan {
   uint8_t* vbad;            // workspace [n_kt][Hkv]
   float cap_lim;            // |scale * q.k| at or below which the softcap polynomial is used
   float k3, k5, k7;         // softcap polynomial coefficients t_n / softcap^(n-1)
+  // The same polynomial in the raw dot product s (u = scale s):
+  // x = s (scale + w (a3 + w (a5 + w a7))), w = s^2, a_n = k_n scale^n, valid
+  // for |s| <= s_lim = cap_lim / |scale|.  cap_raw = 0 when these coefficients
+  // are not normal floats (then the polynomial in u is used).
+  float a3, a5, a7, s_lim;
+  int32_t cap_raw;
   int32_t out_vec;          // output rows may be written with 16-byte stores
   int32_t mask_vec;         // mask rows may be read with 16-byte loads
   int* status;

@@ -150,7 +150,16 @@ struct PfLayout {
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;   // TMEM base address, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
-  static constexpr int THREADS = 320;                    // 10 warps
+  static constexpr int THREADS = 384;                    // 12 warps: 3 warpgroups
+  // Register split (setmaxnreg): the launch gives every thread LAUNCH_REGS;
+  // warpgroup 0 (producer, MMA issuer, two idle warps) drops to LOW_REGS and
+  // the two softmax warpgroups rise to HIGH_REGS.  The total stays within
+  // what the launch holds, so the increase never waits.
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int LOW_REGS = 56;
+  static constexpr int HIGH_REGS = 224;
+  static_assert(128 * LOW_REGS + 256 * HIGH_REGS <= THREADS * LAUNCH_REGS, "register split");
+  static_assert(THREADS * LAUNCH_REGS <= 65536, "launch registers");
   static constexpr uint32_t TMEM_COLS = 512;             // S0, S1 (128 each), O0, O1 (D each)
   static_assert(2 * 128 + 2 * D <= (int)TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory");
@@ -214,15 +223,20 @@ __device__ __forceinline__ void pf_issue_pv(uint32_t d_tmem, uint32_t p_base, ui
   }
 }
 
-// Cell tiles of one row tile in order, skipping the empty ones.
+// Cell tiles of one row tile, skipping the empty ones, from the LAST to the
+// first: under causality the nearest cells come first, and with ALiBi they
+// carry the largest logits, so the running max is set by the first tile and
+// the output rarely needs rescaling afterwards.  All roles walk this order.
 struct PfTiles {
   const uint8_t* cls;    // this row tile's class row [n_kt]
   const uint8_t* vbad;   // [n_kt][Hkv]
   int n_kt, Hkv, g;
-  __device__ __forceinline__ int next(int kt) const {
-    while (kt < n_kt && cls[kt] == kTileSkip) ++kt;
+  __device__ __forceinline__ int below(int kt) const {
+    while (kt >= 0 && cls[kt] == kTileSkip) --kt;
     return kt;
   }
+  __device__ __forceinline__ int first() const { return below(n_kt - 1); }
+  __device__ __forceinline__ int next(int kt) const { return below(kt - 1); }
   __device__ __forceinline__ int code(int kt) const {
     int c = cls[kt];
     if (c == kTileMixed && vbad[(int64_t)kt * Hkv + g]) c = kTileMixedBadV;
@@ -309,6 +323,54 @@ __device__ __forceinline__ void pf_transform_exact(const uint32_t* raw, float* x
   mt = pf_max8(mx);
 }
 
+// Full tiles whose ALiBi bias is linear in the cell index (every cell of the
+// tile at or before every row of the warp, so -slope |row_pos - cell_pos| =
+// C + slope i with C = -slope A), or that carry no ALiBi: packed f32x2
+// arithmetic, two cells per instruction.  The tile is cut into 16 blocks of 8
+// cells; x[i] holds y_i = softcap(scale s_i) + slope (i mod 8), and block m adds
+// off_m = C + 8 slope m (added back by the max here and by the exponent
+// later), which keeps the per-cell ramp to four register pairs.  The softcap
+// polynomial runs in the raw dot product s:
+//   softcap(scale s) = s (scale + w (a3 + w (a5 + w a7))),  w = s^2.
+// Returns the tile max (NaN-propagating) and the largest |s| (range check).
+template <bool CAP, bool ALIBI>
+__device__ __forceinline__ void pf_transform_fast(const uint32_t* raw, float* x, const PrefillPlan& p, float slope,
+                                                  float C, float& mt, float& smax) {
+  const float2 A7 = f2(p.a7), A5 = f2(p.a5), A3 = f2(p.a3), SC = f2(p.lg.scale);
+  float2 R[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) R[q] = ALIBI ? f2(slope * (float)(2 * q), slope * (float)(2 * q + 1)) : f2(0.f);
+  float sm[2] = {0.f, 0.f};
+  float tmax = neg_inf();
+#pragma unroll
+  for (int mb = 0; mb < kPfCells / 8; ++mb) {
+    float bm = neg_inf();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = mb * 8 + 2 * q;
+      const float2 sv = f2(__uint_as_float(raw[i]), __uint_as_float(raw[i + 1]));
+      float2 y;
+      if (CAP) {
+        sm[q & 1] = fmax3(sm[q & 1], fabsf(sv.x), fabsf(sv.y));
+        const float2 w = mul2(sv, sv);
+        float2 h = fma2(w, A7, A5);
+        h = fma2(w, h, A3);
+        const float2 t = fma2(w, h, SC);
+        y = ALIBI ? fma2(sv, t, R[q]) : mul2(sv, t);
+      } else {
+        y = ALIBI ? fma2(sv, SC, R[q]) : mul2(sv, SC);
+      }
+      x[i] = y.x;
+      x[i + 1] = y.y;
+      bm = fmax3_nan(bm, y.x, y.y);
+    }
+    const float off = ALIBI ? fmaf(8.f * slope, (float)mb, C) : 0.f;
+    tmax = fmax_nan(tmax, bm + off);
+  }
+  mt = tmax;
+  smax = fmaxf(sm[0], sm[1]);
+}
+
 // Mixed tiles: per-cell visibility (range, sequence, causal, mask != -inf)
 // and the mask bias; excluded cells become -inf and lose their bit in vis.
 // With explicit cell positions the ALiBi term is added here (the transform
@@ -392,6 +454,43 @@ __device__ __forceinline__ void pf_store32(const OutSpec& o, int64_t i0, const f
   }
 }
 
+// Lazy rescaling of the running state (m, l) by the tile max mt, then the
+// weights p_i = 2^((x_i + off_m) log2 e - m log2 e) of one row of a tile, their
+// sum into l, and P packed to 16 bits.  Block m of 8 cells adds the offset
+// off_m = boff + bstep m (nonzero on the fast ALiBi path only), folded into
+// one exponent bias per block.  The max is only raised when it grows by more
+// than ln 256, so the weights stay below 256 and O is rescaled rarely.
+template <typename KT>
+__device__ __forceinline__ void pf_weights(const float* x, float boff, float bstep, float mt, float& m, float& l,
+                                           float& mneg2, uint32_t* pk, bool& need, float& factor) {
+  constexpr float kLazy = 5.545177444479562f;   // ln 256
+  need = !(mt <= m + kLazy);   // NaN compares false: a NaN max always rescales
+  factor = 1.f;
+  if (need) {
+    const float mn = fmax_nan(m, mt);
+    factor = ex2((m - mn) * kLog2e);        // 0 when m was -inf
+    l *= factor;
+    m = mn;
+    mneg2 = (m == neg_inf()) ? 0.f : -m * kLog2e;
+  }
+  float2 ls[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
+  const float2 L2E = f2(kLog2e);
+#pragma unroll
+  for (int mb = 0; mb < kPfCells / 8; ++mb) {
+    const float2 E = f2(fmaf(fmaf(bstep, (float)mb, boff), kLog2e, mneg2));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = mb * 8 + 2 * q;
+      const float2 a = fma2(f2(x[i], x[i + 1]), L2E, E);
+      const float p0 = ex2(a.x), p1 = ex2(a.y);
+      ls[q] = add2(ls[q], f2(p0, p1));
+      pk[i / 2] = pf_pack<KT>(p0, p1);
+    }
+  }
+  const float2 s4 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
+  l += s4.x + s4.y;
+}
+
 template <typename KT, int D>
 __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& tiles, unsigned char* sm,
                                            uint64_t* bars, volatile int* abort_flag, uint32_t tmem, int rt,
@@ -419,76 +518,82 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
   const uint32_t tO = lane_base + 256u + (uint32_t)slot * D;
   unsigned char* Ps = sm + L::OFF_P + slot * L::PTILE;
   const float* mrow = (p.f.mask && rvalid) ? p.f.mask + (int64_t)r * p.f.mask_sr : nullptr;
-  constexpr float kLazy = 5.545177444479562f;   // ln 256: rescale only when the max grows by more
 
   float m = neg_inf(), l = 0.f, mneg2 = 0.f;    // mneg2 = -m * log2(e) (0 while m = -inf)
   int j = 0;
   bool ok = true;
-  for (int kt = tiles.next(0); kt < tiles.n_kt; kt = tiles.next(kt + 1), ++j) {
+  for (int kt = tiles.first(); kt >= 0; kt = tiles.next(kt), ++j) {
     const int code = tiles.code(kt);
     if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
     tc_fence_after();
-    uint32_t raw[kPfCells];
-#pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
-    tmem_wait_ld();
-
-    float x[kPfCells];
     uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
-    float mt, umax = 0.f;
+    uint32_t pk[kPfCells / 2];   // P of this row, packed to 16 bits
+    bool need;                    // the running max grew: O needs rescaling
+    float factor;                 // ... by this factor
     const int c0 = kt * kPfCells;
     const float A = (float)(rv.rp + rv.rb - c0);
-    const int32_t* cpos = p.f.cell_pos ? p.f.cell_pos + c0 : nullptr;
-    // full tiles: ALiBi in the transform; mixed tiles with explicit positions:
-    // in the visibility pass (cell_pos may end inside the tile)
-    const int al_t = (code == kTileFull || al == 1) ? al : 0;
-    switch ((cap ? 3 : 0) + al_t) {
-      case 0: pf_transform<false, 0>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
-      case 1: pf_transform<false, 1>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
-      case 2: pf_transform<false, 2>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
-      case 3: pf_transform<true, 0>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
-      case 4: pf_transform<true, 1>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
-      default: pf_transform<true, 2>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
-    }
-    if (cap && __any_sync(0xffffffffu, !(umax <= p.cap_lim))) {
-      // some logit outside the polynomial's range: redo the row from S
+    // Packed fast path: a full tile with no ALiBi, or with affine positions and
+    // every cell at or before every row of the warp (see pf_transform_fast).
+    // Each path below reads S, computes the logits and then the weights on
+    // its own, so only P crosses the join (it keeps register use low).
+    bool fast = code == kTileFull && (!cap || p.cap_raw) &&
+                (al == 0 || (al == 1 && __all_sync(0xffffffffu, !rvalid || A >= (float)(kPfCells - 1))));
+    if (fast) {
+      uint32_t raw[kPfCells];
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
       tmem_wait_ld();
-      if (al_t == 0) pf_transform_exact<0>(raw, x, p, nslope, A, rpf, cpos, mt);
-      else if (al_t == 1) pf_transform_exact<1>(raw, x, p, nslope, A, rpf, cpos, mt);
-      else pf_transform_exact<2>(raw, x, p, nslope, A, rpf, cpos, mt);
+      const float slope = -nslope, C = nslope * A;
+      float x[kPfCells], mt, smax = 0.f;
+      if (cap) {
+        if (al == 1) pf_transform_fast<true, true>(raw, x, p, slope, C, mt, smax);
+        else pf_transform_fast<true, false>(raw, x, p, slope, C, mt, smax);
+      } else {
+        if (al == 1) pf_transform_fast<false, true>(raw, x, p, slope, C, mt, smax);
+        else pf_transform_fast<false, false>(raw, x, p, slope, C, mt, smax);
+      }
+      // outside the polynomial's range: the tile goes to the scalar path
+      // below, which reads S from tensor memory again
+      if (cap && __any_sync(0xffffffffu, !(smax <= p.s_lim))) {
+        fast = false;
+      } else {
+        tc_fence_before();
+        mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
+        pf_weights<KT>(x, al == 1 ? C : 0.f, al == 1 ? 8.f * slope : 0.f, mt, m, l, mneg2, pk, need, factor);
+      }
     }
-    tc_fence_before();
-    mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
-    if (code != kTileFull) pf_visibility(x, vis, p, rv, rvalid, c0, mrow, mask_vec, al == 2, nslope, mt);
-
-    // lazy rescaling of the running state
-    const bool need = !(mt <= m + kLazy);   // NaN compares false: a NaN max always rescales
-    float factor = 1.f;
-    if (need) {
-      const float mn = fmax_nan(m, mt);
-      factor = ex2((m - mn) * kLog2e);        // 0 when m was -inf
-      l *= factor;
-      m = mn;
-      mneg2 = (m == neg_inf()) ? 0.f : -m * kLog2e;
-    }
-
-    // Weights, their sum, and P packed to 16 bits (64 registers instead of
-    // 128 while O is rescaled below).
-    float ls[8];
+    if (!fast) {
+      const int32_t* cpos = p.f.cell_pos ? p.f.cell_pos + c0 : nullptr;
+      // full tiles: ALiBi in the transform; mixed tiles with explicit
+      // positions: in the visibility pass (cell_pos may end inside the tile)
+      const int al_t = (code == kTileFull || al == 1) ? al : 0;
+      uint32_t raw[kPfCells];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) ls[k] = 0.f;
-    uint32_t pk[kPfCells / 2];
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
+      tmem_wait_ld();
+      float x[kPfCells], mt, umax = 0.f;
+      switch ((cap ? 3 : 0) + al_t) {
+        case 0: pf_transform<false, 0>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+        case 1: pf_transform<false, 1>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+        case 2: pf_transform<false, 2>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+        case 3: pf_transform<true, 0>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+        case 4: pf_transform<true, 1>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+        default: pf_transform<true, 2>(raw, x, scale, p.k3, p.k5, p.k7, nslope, A, rpf, cpos, mt, umax); break;
+      }
+      if (cap && __any_sync(0xffffffffu, !(umax <= p.cap_lim))) {
+        // some logit outside the polynomial's range: redo the row from S
 #pragma unroll
-    for (int i = 0; i < kPfCells; i += 2) {
-      const float p0 = ex2(fmaf(x[i], kLog2e, mneg2));
-      const float p1 = ex2(fmaf(x[i + 1], kLog2e, mneg2));
-      ls[(i >> 1) & 7] += p0;
-      ls[(i >> 1) & 7] += p1;
-      pk[i / 2] = pf_pack<KT>(p0, p1);
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
+        tmem_wait_ld();
+        if (al_t == 0) pf_transform_exact<0>(raw, x, p, nslope, A, rpf, cpos, mt);
+        else if (al_t == 1) pf_transform_exact<1>(raw, x, p, nslope, A, rpf, cpos, mt);
+        else pf_transform_exact<2>(raw, x, p, nslope, A, rpf, cpos, mt);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
+      if (code != kTileFull) pf_visibility(x, vis, p, rv, rvalid, c0, mrow, mask_vec, al == 2, nslope, mt);
+      pf_weights<KT>(x, 0.f, 0.f, mt, m, l, mneg2, pk, need, factor);
     }
-    l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
 
     // P V of the previous tile must be complete before its P buffer is
     // overwritten and before O is rescaled.
@@ -502,8 +607,13 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
         uint32_t o[32];
         tmem_ld32(tO + ch * 32, o);
         tmem_wait_ld();
+        const float2 F = f2(factor);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+        for (int e = 0; e < 32; e += 2) {
+          const float2 v = mul2(f2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), F);
+          o[e] = __float_as_uint(v.x);
+          o[e + 1] = __float_as_uint(v.y);
+        }
         tmem_st32(tO + ch * 32, o);
       }
       tmem_wait_st();
@@ -659,14 +769,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const PfTiles tiles{p.cls + (int64_t)rt * p.n_kt, p.vbad, p.n_kt, p.Hkv, g};
 
+  if (warp >= 4) {
+    // ---- softmax warpgroups ----
+    setmaxnreg_inc<L::HIGH_REGS>();
+    const int slot = (warp >> 2) - 1;
+    if (slot < n_slots)
+      pf_softmax<KT, D>(p, tiles, sm, bars, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane);
+  } else {
+  setmaxnreg_dec<L::LOW_REGS>();
   if (warp == 0) {
     // ---- TMA producer ----
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
-      int kt = tiles.next(0);
+      int kt = tiles.first();
       int64_t Lc = 0;   // loads issued into the ring
       bool ok = true;
-      const bool any = kt < p.n_kt;
+      const bool any = kt >= 0;
       if (any) {
         mbar_arrive_expect_tx(q_full, (uint32_t)(n_slots * L::TILE));
         for (int s = 0; s < n_slots; ++s)
@@ -675,7 +793,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, q_full, bx * 64, h0 + s, rt * kPfRows,
                         pol);
       }
-      for (; ok && kt < p.n_kt; kt = tiles.next(kt + 1)) {
+      for (; ok && kt >= 0; kt = tiles.next(kt)) {
         for (int kv = 0; kv < 2; ++kv) {
           const int st = (int)(Lc % NS);
           if (Lc >= NS && !pf_wait(&kv_empty[st], (uint32_t)(((Lc / NS) + 1) & 1), p.status, abort_flag)) {
@@ -703,8 +821,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t idO = umma_idesc_f16(kPfRows, D, bf, 0, 1);
       const uint32_t q_addr = smem_u32(sm + L::OFF_Q), p_addr = smem_u32(sm + L::OFF_P);
       const uint32_t kv_addr = smem_u32(sm + L::OFF_KV);
-      int kt = tiles.next(0);
-      bool ok = kt < p.n_kt;
+      int kt = tiles.first();
+      bool ok = kt >= 0;
       if (ok) {
         ok = pf_wait(q_full, 0, p.status, abort_flag) && pf_wait(&kv_full[0], 0, p.status, abort_flag);
         if (ok) {
@@ -716,9 +834,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           umma_commit(&kv_empty[0]);
         }
       }
-      for (int64_t j = 0; ok && kt < p.n_kt; ++j) {
-        const int kn = tiles.next(kt + 1);
-        const bool has_next = kn < p.n_kt;
+      for (int64_t j = 0; ok && kt >= 0; ++j) {
+        const int kn = tiles.next(kt);
+        const bool has_next = kn >= 0;
         const bool pv_mma = tiles.code(kt) != kTileMixedBadV;
         const int64_t LK = 2 * (j + 1), LV = 2 * j + 1;
         const int stK = (int)(LK % NS), stV = (int)(LV % NS);
@@ -746,11 +864,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       umma_commit(mma_done);   // arrives once every MMA issued above has retired
     }
-  } else {
-    // ---- softmax warpgroups ----
-    const int slot = (warp - 2) >> 2;
-    if (slot < n_slots)
-      pf_softmax<KT, D>(p, tiles, sm, bars, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane);
+  }   // warps 2 and 3 have no role
   }
 
   tc_fence_before();

@@ -18,6 +18,18 @@
 
 namespace attn {
 
+// ---- register reallocation between warpgroups ----------------------------------
+// Every warp of a warpgroup must execute the same one; the sum over the CTA
+// must stay within the registers the launch reserved.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---- descriptors -------------------------------------------------------------
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2).
