@@ -352,7 +352,7 @@ int32_t check_prefill(const attn_args* a) {
 }
 
 struct PrefillWs {
-  size_t vbad_off, total;
+  size_t vbad_off, kn2_off, total;
 };
 
 PrefillWs prefill_ws_layout(const attn_args* a) {
@@ -360,7 +360,8 @@ PrefillWs prefill_ws_layout(const attn_args* a) {
   const size_t n_kt = ((size_t)a->n_cells + kPfTile - 1) / kPfTile;
   PrefillWs w;
   w.vbad_off = align256(n_rt * n_kt);
-  w.total = w.vbad_off + align256(n_kt * a->n_head_kv);
+  w.kn2_off = w.vbad_off + align256(n_kt * a->n_head_kv);
+  w.total = w.kn2_off + align256(n_kt * a->n_head_kv * sizeof(float));
   return w;
 }
 
@@ -610,7 +611,7 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   PrefillPlan p{};
   p.R = a->n_rows; p.Hq = a->n_head_q; p.Hkv = a->n_head_kv; p.G = a->n_head_q / a->n_head_kv;
   p.D = a->head_dim; p.N = a->n_cells; p.kv_type = a->kv_type;
-  p.v = a->v; p.kv_sc = a->kv_stride_cell; p.kv_sh = a->kv_stride_head;
+  p.k = a->k; p.v = a->v; p.kv_sc = a->kv_stride_cell; p.kv_sh = a->kv_stride_head;
   p.out = OutSpec{a->out, a->out_type, a->o_stride_row, a->o_stride_head};
   p.f = RowFilter{a->row_begin, a->row_end, a->cell_seq, a->row_seq, a->cell_pos, a->row_pos,
                   a->causal, a->mask, a->mask_stride_row};
@@ -621,6 +622,7 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   char* wsb = static_cast<char*>(ws);
   p.cls = reinterpret_cast<uint8_t*>(wsb);
   p.vbad = reinterpret_cast<uint8_t*>(wsb + wl.vbad_off);
+  p.kn2 = reinterpret_cast<float*>(wsb + wl.kn2_off);
   // Softcap polynomial: x = u + u w (k3 + w (k5 + w k7)), w = u^2, the odd
   // Taylor series of c tanh(u / c) through u^7, used for |u| <= c / 5.
   if (a->softcap > 0.f) {
@@ -629,17 +631,26 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
     p.k3 = (float)(-1.0 / (3.0 * c2));
     p.k5 = (float)(2.0 / (15.0 * c2 * c2));
     p.k7 = (float)(-17.0 / (315.0 * c2 * c2 * c2));
+    // tanh y = y - y^3/3 + 2 y^5/15 - 17 y^7/315 + 62 y^9/2835 - ...
     const double sc = a->scale, s2 = sc * sc;
-    const double a3 = p.k3 * sc * s2, a5 = p.k5 * sc * s2 * s2, a7 = p.k7 * sc * s2 * s2 * s2;
+    const double a3 = -1.0 / 3.0 / c2 * sc * s2;
+    const double a5 = 2.0 / 15.0 / (c2 * c2) * sc * s2 * s2;
+    const double a7 = -17.0 / 315.0 / (c2 * c2 * c2) * sc * s2 * s2 * s2;
+    const double a9 = 62.0 / 2835.0 / (c2 * c2 * c2 * c2) * sc * s2 * s2 * s2 * s2;
+    const double s_lim = 0.4 * c / std::fabs(sc);
     auto normal = [](double v) { return std::fabs(v) >= 1.1754943508222875e-38 && std::fabs(v) <= 3.0e38; };
-    if (sc != 0.0 && std::isfinite(sc) && normal(a3) && normal(a5) && normal(a7) && normal(0.2 * c / std::fabs(sc))) {
+    if (sc != 0.0 && std::isfinite(sc) && normal(a3) && normal(a5) && normal(a7) && normal(a9) &&
+        normal(s_lim) && normal(s_lim * s_lim)) {
       p.a3 = (float)a3;
       p.a5 = (float)a5;
       p.a7 = (float)a7;
-      p.s_lim = (float)(0.2 * c / std::fabs(sc));
+      p.a9 = (float)a9;
+      p.s_lim = (float)s_lim;
+      p.bound2 = (float)(0.998 * s_lim * s_lim);
       p.cap_raw = 1;
     }
   }
+  if (!p.cap_raw) p.kn2 = nullptr;   // the tile norms serve the packed softcap only
   const int oes = dtype_size(a->out_type);
   const int64_t ovec = 16 / oes;
   p.out_vec = aligned16(a->out) && (a->n_rows <= 1 || a->o_stride_row % ovec == 0) &&

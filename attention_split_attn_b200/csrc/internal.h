@@ -116,6 +116,7 @@ enum : uint8_t { kTileSkip = 0, kTileFull = 1, kTileMixed = 2, kTileMixedBadV = 
 struct PrefillPlan {
   int32_t R, Hq, Hkv, G, D, N;
   int32_t kv_type;
+  const void* k;            // K cache (tile norms for the softcap range bound)
   const void* v;            // V cache (scanned for non-finite values)
   int64_t kv_sc, kv_sh;     // its cell and head strides (elements)
   OutSpec out;
@@ -127,12 +128,17 @@ struct PrefillPlan {
   uint8_t* vbad;            // workspace [n_kt][Hkv]
   float cap_lim;            // |scale * q.k| at or below which the softcap polynomial is used
   float k3, k5, k7;         // softcap polynomial coefficients t_n / softcap^(n-1)
-  // The same polynomial in the raw dot product s (u = scale s):
-  // x = s (scale + w (a3 + w (a5 + w a7))), w = s^2, a_n = k_n scale^n, valid
-  // for |s| <= s_lim = cap_lim / |scale|.  cap_raw = 0 when these coefficients
-  // are not normal floats (then the polynomial in u is used).
-  float a3, a5, a7, s_lim;
+  // Packed path: the odd Taylor series of c tanh(u / c) through u^9 in the raw
+  // dot product s (u = scale s): x = s (scale + w (a3 + w (a5 + w (a7 + w a9)))),
+  // w = s^2, a_n = t_n scale^n / c^(n-1); truncation below 3.7e-7 c for
+  // |u| <= 0.4 c, i.e. |s| <= s_lim.  cap_raw = 0 when these coefficients are
+  // not normal floats (then the scalar path's polynomial in u is used).
+  float a3, a5, a7, a9, s_lim;
   int32_t cap_raw;
+  // A tile needs no per-cell range check when |s| <= |q| |k| is within s_lim
+  // for every row: |q_r|^2 max_c |k_c|^2 <= bound2 (= 0.998 s_lim^2).
+  float bound2;
+  float* kn2;               // workspace [n_kt][Hkv]: max |k_c|^2 over the tile (NaN/inf kept)
   int32_t out_vec;          // output rows may be written with 16-byte stores
   int32_t mask_vec;         // mask rows may be read with 16-byte loads
   int* status;

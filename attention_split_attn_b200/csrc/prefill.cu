@@ -128,6 +128,45 @@ __global__ void __launch_bounds__(256) prefill_classify_kernel(PrefillPlan p) {
     }
     const int any_bad = __syncthreads_or(bad ? 1 : 0);
     if (tid == 0) p.vbad[(int64_t)kt * p.Hkv + g] = any_bad ? 1 : 0;
+    if (p.kn2) {
+      // max over the tile's cells of |k_c|^2 (NaN-propagating: a non-finite K
+      // makes the bound fail).  The per_row chunks of one cell sit in
+      // per_row consecutive lanes (per_row divides 32 and 256).
+      __shared__ float wmax[8];
+      float mx = 0.f;
+      for (int i = tid; i < kPfCells * per_row; i += 256) {
+        const int c = kt * kPfCells + i / per_row;
+        float ss = 0.f;
+        if (c < p.N) {
+          const uint16_t* row = static_cast<const uint16_t*>(p.k) + (int64_t)c * p.kv_sc + (int64_t)g * p.kv_sh;
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + (i % per_row));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float lo, hi;
+            if (p.kv_type == ATTN_BF16) {
+              lo = __uint_as_float(ws[k] << 16);
+              hi = __uint_as_float(ws[k] & 0xffff0000u);
+            } else {
+              lo = __half2float(__ushort_as_half((unsigned short)(ws[k] & 0xffffu)));
+              hi = __half2float(__ushort_as_half((unsigned short)(ws[k] >> 16)));
+            }
+            ss = fmaf(lo, lo, ss);
+            ss = fmaf(hi, hi, ss);
+          }
+        }
+        for (int o = per_row / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        mx = fmax_nan(mx, ss);
+      }
+      for (int o = 16; o > 0; o >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if ((tid & 31) == 0) wmax[tid >> 5] = mx;
+      __syncthreads();
+      if (tid == 0) {
+        float m = wmax[0];
+        for (int w8 = 1; w8 < 8; ++w8) m = fmax_nan(m, wmax[w8]);
+        p.kn2[(int64_t)kt * p.Hkv + g] = m;
+      }
+    }
   }
 }
 
@@ -330,13 +369,15 @@ __device__ __forceinline__ void pf_transform_exact(const uint32_t* raw, float* x
 // cells; x[i] holds y_i = softcap(scale s_i) + slope (i mod 8), and block m adds
 // off_m = C + 8 slope m (added back by the max here and by the exponent
 // later), which keeps the per-cell ramp to four register pairs.  The softcap
-// polynomial runs in the raw dot product s:
-//   softcap(scale s) = s (scale + w (a3 + w (a5 + w a7))),  w = s^2.
-// Returns the tile max (NaN-propagating) and the largest |s| (range check).
-template <bool CAP, bool ALIBI>
+// is the odd Taylor polynomial through u^9 in the raw dot product s:
+//   softcap(scale s) = s (scale + w (a3 + w (a5 + w (a7 + w a9)))),  w = s^2.
+// CAPM: 0 no softcap; 1 softcap with a per-cell range check (returns the
+// largest |s| in smax); 2 softcap on a tile whose range the caller has
+// bounded (|s| <= |q| |k| <= s_lim).  Returns the tile max (NaN-propagating).
+template <int CAPM, bool ALIBI>
 __device__ __forceinline__ void pf_transform_fast(const uint32_t* raw, float* x, const PrefillPlan& p, float slope,
                                                   float C, float& mt, float& smax) {
-  const float2 A7 = f2(p.a7), A5 = f2(p.a5), A3 = f2(p.a3), SC = f2(p.lg.scale);
+  const float2 A9 = f2(p.a9), A7 = f2(p.a7), A5 = f2(p.a5), A3 = f2(p.a3), SC = f2(p.lg.scale);
   float2 R[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) R[q] = ALIBI ? f2(slope * (float)(2 * q), slope * (float)(2 * q + 1)) : f2(0.f);
@@ -350,10 +391,11 @@ __device__ __forceinline__ void pf_transform_fast(const uint32_t* raw, float* x,
       const int i = mb * 8 + 2 * q;
       const float2 sv = f2(__uint_as_float(raw[i]), __uint_as_float(raw[i + 1]));
       float2 y;
-      if (CAP) {
-        sm[q & 1] = fmax3(sm[q & 1], fabsf(sv.x), fabsf(sv.y));
+      if (CAPM > 0) {
+        if (CAPM == 1) sm[q & 1] = fmax3(sm[q & 1], fabsf(sv.x), fabsf(sv.y));
         const float2 w = mul2(sv, sv);
-        float2 h = fma2(w, A7, A5);
+        float2 h = fma2(w, A9, A7);
+        h = fma2(w, h, A5);
         h = fma2(w, h, A3);
         const float2 t = fma2(w, h, SC);
         y = ALIBI ? fma2(sv, t, R[q]) : mul2(sv, t);
@@ -522,10 +564,30 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
   float m = neg_inf(), l = 0.f, mneg2 = 0.f;    // mneg2 = -m * log2(e) (0 while m = -inf)
   int j = 0;
   bool ok = true;
+  float qn2 = 0.f;   // |q_r|^2 of this row and head (softcap range bound)
   for (int kt = tiles.first(); kt >= 0; kt = tiles.next(kt), ++j) {
     const int code = tiles.code(kt);
     if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
     tc_fence_after();
+    if (j == 0 && cap && p.kn2) {
+      // the Q tile is resident (its load completed before the first S)
+      if (!pf_wait_warp(&bars[0], 0u, p.status, abort_flag)) { ok = false; break; }
+      const unsigned char* Qs = sm + L::OFF_Q + slot * L::TILE;
+      float a = 0.f, b = 0.f;
+#pragma unroll
+      for (int k8 = 0; k8 < D / 8; ++k8) {
+        const uint32_t off = (uint32_t)(k8 >> 3) * L::BOX + (uint32_t)row_t * 128u +
+                             ((uint32_t)((k8 & 7) ^ (row_t & 7)) << 4);
+        float v[8];
+        unpack_vec<KT>(*reinterpret_cast<const uint4*>(Qs + off), v);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          a = fmaf(v[e], v[e], a);
+          b = fmaf(v[e + 1], v[e + 1], b);
+        }
+      }
+      qn2 = a + b;
+    }
     uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
     uint32_t pk[kPfCells / 2];   // P of this row, packed to 16 bits
     bool need;                    // the running max grew: O needs rescaling
@@ -545,16 +607,22 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       tmem_wait_ld();
       const float slope = -nslope, C = nslope * A;
       float x[kPfCells], mt, smax = 0.f;
-      if (cap) {
-        if (al == 1) pf_transform_fast<true, true>(raw, x, p, slope, C, mt, smax);
-        else pf_transform_fast<true, false>(raw, x, p, slope, C, mt, smax);
+      // every row's |q|^2 max |k|^2 within range: no per-cell check
+      const bool bounded = cap && p.kn2 != nullptr &&
+                           __all_sync(0xffffffffu, qn2 * __ldg(p.kn2 + (int64_t)kt * p.Hkv + tiles.g) <= p.bound2);
+      if (bounded) {
+        if (al == 1) pf_transform_fast<2, true>(raw, x, p, slope, C, mt, smax);
+        else pf_transform_fast<2, false>(raw, x, p, slope, C, mt, smax);
+      } else if (cap) {
+        if (al == 1) pf_transform_fast<1, true>(raw, x, p, slope, C, mt, smax);
+        else pf_transform_fast<1, false>(raw, x, p, slope, C, mt, smax);
       } else {
-        if (al == 1) pf_transform_fast<false, true>(raw, x, p, slope, C, mt, smax);
-        else pf_transform_fast<false, false>(raw, x, p, slope, C, mt, smax);
+        if (al == 1) pf_transform_fast<0, true>(raw, x, p, slope, C, mt, smax);
+        else pf_transform_fast<0, false>(raw, x, p, slope, C, mt, smax);
       }
       // outside the polynomial's range: the tile goes to the scalar path
       // below, which reads S from tensor memory again
-      if (cap && __any_sync(0xffffffffu, !(smax <= p.s_lim))) {
+      if (cap && !bounded && __any_sync(0xffffffffu, !(smax <= p.s_lim))) {
         fast = false;
       } else {
         tc_fence_before();
@@ -843,6 +911,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (has_next && !pf_wait(&kv_full[stK], (uint32_t)((LK / NS) & 1), p.status, abort_flag)) break;
         if (!pf_wait(&kv_full[stV], (uint32_t)((LV / NS) & 1), p.status, abort_flag)) break;
         tc_fence_after();
+        // per head: the next tile's scores as soon as the softmax has read
+        // this tile's S, then this tile's P V
         for (int s = 0; s < n_slots && ok; ++s) {
           if (has_next) {
             if (!pf_wait(&s_free[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
