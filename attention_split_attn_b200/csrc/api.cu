@@ -352,7 +352,7 @@ int32_t check_prefill(const attn_args* a) {
 }
 
 struct PrefillWs {
-  size_t vbad_off, kn2_off, total;
+  size_t vbad_off, kn2_off, bits_off, total;
 };
 
 PrefillWs prefill_ws_layout(const attn_args* a) {
@@ -361,7 +361,10 @@ PrefillWs prefill_ws_layout(const attn_args* a) {
   PrefillWs w;
   w.vbad_off = align256(n_rt * n_kt);
   w.kn2_off = w.vbad_off + align256(n_kt * a->n_head_kv);
-  w.total = w.kn2_off + align256(n_kt * a->n_head_kv * sizeof(float));
+  w.bits_off = w.kn2_off + align256(n_kt * a->n_head_kv * sizeof(float));
+  // visibility bits of every tile when a mask is given (1/32 of the mask's size)
+  const size_t bits = a->mask ? n_rt * n_kt * (size_t)kPfTile * 16 : 0;
+  w.total = w.bits_off + align256(bits);
   return w;
 }
 
@@ -623,6 +626,7 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   p.cls = reinterpret_cast<uint8_t*>(wsb);
   p.vbad = reinterpret_cast<uint8_t*>(wsb + wl.vbad_off);
   p.kn2 = reinterpret_cast<float*>(wsb + wl.kn2_off);
+  p.bits = a->mask ? reinterpret_cast<uint32_t*>(wsb + wl.bits_off) : nullptr;
   // Softcap polynomial: x = u + u w (k3 + w (k5 + w k7)), w = u^2, the odd
   // Taylor series of c tanh(u / c) through u^7, used for |u| <= c / 5.
   if (a->softcap > 0.f) {

@@ -108,10 +108,17 @@ cudaError_t launch_selected(const SelectedPlan& p, cudaStream_t stream);
 // ---- causal prefill -----------------------------------------------------------
 // Tiles of 128 query rows x 128 cells.  A classifier kernel tags every (row
 // tile, cell tile) as skipped (no row sees any cell), full (every row sees
-// every cell and the mask adds exactly 0 there) or mixed, and every (cell
-// tile, KV head) whose V holds a non-finite value; the tensor-core kernel then
+// every cell and the mask adds exactly 0 there), bits (with a mask: the mask
+// adds exactly 0 on every visible cell, so the visibility bits the classifier
+// stores say everything) or mixed (visible cells with a nonzero mask value),
+// plus a flag for a visible cell after its row's position; and every (cell
+// tile, KV head) whose V holds a non-finite value.  The tensor-core kernel then
 // runs one CTA per (row tile, pair of q heads of one KV group).
-enum : uint8_t { kTileSkip = 0, kTileFull = 1, kTileMixed = 2, kTileMixedBadV = 3 };
+enum : uint8_t {
+  kTileSkip = 0, kTileFull = 1, kTileMixed = 2, kTileBits = 3,   // stored class (low 2 bits)
+  kTileLate = 8,                                                  // stored flag
+  kTileMixedBadV = 4                                              // kernel-side code only
+};
 
 struct PrefillPlan {
   int32_t R, Hq, Hkv, G, D, N;
@@ -125,6 +132,7 @@ struct PrefillPlan {
   int32_t n_rt, n_kt;       // row tiles, cell tiles (128 each)
   int32_t n_pairs;          // ceil(G / 2): CTAs per (row tile, KV head)
   uint8_t* cls;             // workspace [n_rt][n_kt]
+  uint32_t* bits;           // workspace [n_rt][n_kt][128 rows][4 words] (with a mask) or NULL
   uint8_t* vbad;            // workspace [n_kt][Hkv]
   float cap_lim;            // |scale * q.k| at or below which the softcap polynomial is used
   float k3, k5, k7;         // softcap polynomial coefficients t_n / softcap^(n-1)

@@ -86,16 +86,16 @@ __global__ void __launch_bounds__(256) prefill_classify_kernel(PrefillPlan p) {
     const bool cin = c < p.N;
     const int32_t cs = (cin && p.f.cell_seq) ? __ldg(p.f.cell_seq + c) : 0;
     const int32_t cpos_given = (cin && p.f.cell_pos) ? __ldg(p.f.cell_pos + c) : 0;
-    bool any = false, notfull = false;
+    bool any = false, notfull = false, bias = false, late = false;
     const int r_end = min(p.R, (rt + 1) * kPfRows);
+    // every warp walks the same rows (its 32 cells of one row per step), so
+    // its ballot is one 32-bit word of that row's visibility bits
     for (int r = rt * kPfRows + (tid >> 7); r < r_end; r += 2) {
       const RowVis rv = row_vis(p.f, r, p.N);
       bool vis = cin && c >= rv.rb && c < rv.re;
       if (p.f.cell_seq) vis = vis && cs == rv.rs;
-      if (p.f.causal) {
-        const int32_t cp = p.f.cell_pos ? cpos_given : c - rv.rb;
-        vis = vis && cp <= rv.rp;
-      }
+      const int32_t cp = p.f.cell_pos ? cpos_given : c - rv.rb;
+      if (p.f.causal) vis = vis && cp <= rv.rp;
       bool zero_bias = true;
       if (p.f.mask && vis) {
         const float mv = __ldg(p.f.mask + (int64_t)r * p.f.mask_sr + c);
@@ -104,10 +104,22 @@ __global__ void __launch_bounds__(256) prefill_classify_kernel(PrefillPlan p) {
       }
       any |= vis;
       notfull |= !(vis && zero_bias);
+      bias |= vis && !zero_bias;
+      late |= vis && cp > rv.rp;
+      if (p.bits) {
+        const uint32_t word = __ballot_sync(0xffffffffu, vis);
+        if ((tid & 31) == 0)
+          p.bits[((b * kPfRows + (r - rt * kPfRows)) << 2) + ((tid & 127) >> 5)] = word;
+      }
     }
     const int a = __syncthreads_or(any ? 1 : 0);
     const int nf = __syncthreads_or(notfull ? 1 : 0);
-    if (tid == 0) p.cls[b] = !a ? kTileSkip : (nf ? kTileMixed : kTileFull);
+    const int bs = __syncthreads_or(bias ? 1 : 0);
+    const int lt = __syncthreads_or(late ? 1 : 0);
+    if (tid == 0) {
+      const int cl = !a ? kTileSkip : !nf ? kTileFull : (p.bits && !bs) ? kTileBits : kTileMixed;
+      p.cls[b] = (uint8_t)(cl | (lt ? kTileLate : 0));
+    }
   } else {
     const int64_t vb = b - n_cls;
     const int kt = (int)(vb / p.Hkv), g = (int)(vb % p.Hkv);
@@ -271,16 +283,20 @@ struct PfTiles {
   const uint8_t* vbad;   // [n_kt][Hkv]
   int n_kt, Hkv, g;
   __device__ __forceinline__ int below(int kt) const {
-    while (kt >= 0 && cls[kt] == kTileSkip) --kt;
+    while (kt >= 0 && (cls[kt] & 3) == kTileSkip) --kt;
     return kt;
   }
   __device__ __forceinline__ int first() const { return below(n_kt - 1); }
   __device__ __forceinline__ int next(int kt) const { return below(kt - 1); }
+  // Full, Mixed or Bits; MixedBadV for a non-full tile whose V (this KV head)
+  // holds a non-finite value (P V then runs on the CUDA cores).
   __device__ __forceinline__ int code(int kt) const {
-    int c = cls[kt];
-    if (c == kTileMixed && vbad[(int64_t)kt * Hkv + g]) c = kTileMixedBadV;
+    const int c = cls[kt] & 3;
+    if (c >= kTileMixed && vbad[(int64_t)kt * Hkv + g]) return kTileMixedBadV;
     return c;
   }
+  __device__ __forceinline__ bool bits(int kt) const { return (cls[kt] & 3) == kTileBits; }
+  __device__ __forceinline__ bool late(int kt) const { return (cls[kt] & kTileLate) != 0; }
 };
 
 // ---------------------------------------------------------------------------
@@ -411,6 +427,27 @@ __device__ __forceinline__ void pf_transform_fast(const uint32_t* raw, float* x,
   }
   mt = tmax;
   smax = fmaxf(sm[0], sm[1]);
+}
+
+// Bits tiles on the packed path: cells whose visibility bit is clear become
+// -inf (whatever their logit, NaN included), and the tile max is taken again
+// over the visible cells, block offsets included.
+__device__ __forceinline__ void pf_apply_bits(float* x, const uint32_t* vis, float boff, float bstep, float& mt) {
+  float tmax = neg_inf();
+#pragma unroll
+  for (int mb = 0; mb < kPfCells / 8; ++mb) {
+    const uint32_t w = vis[mb >> 2] >> ((mb & 3) * 8);
+    float bm = neg_inf();
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const int i = mb * 8 + e;
+      x[i] = ((w >> e) & 1u) ? x[i] : neg_inf();
+      x[i + 1] = ((w >> (e + 1)) & 1u) ? x[i + 1] : neg_inf();
+      bm = fmax3_nan(bm, x[i], x[i + 1]);
+    }
+    tmax = fmax_nan(tmax, bm + fmaf(bstep, (float)mb, boff));
+  }
+  mt = tmax;
 }
 
 // Mixed tiles: per-cell visibility (range, sequence, causal, mask != -inf)
@@ -594,12 +631,13 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     float factor;                 // ... by this factor
     const int c0 = kt * kPfCells;
     const float A = (float)(rv.rp + rv.rb - c0);
-    // Packed fast path: a full tile with no ALiBi, or with affine positions and
-    // every cell at or before every row of the warp (see pf_transform_fast).
+    // Packed fast path: a full or bits tile with no ALiBi, or with affine
+    // positions and no visible cell after its row (see pf_transform_fast).
     // Each path below reads S, computes the logits and then the weights on
     // its own, so only P crosses the join (it keeps register use low).
-    bool fast = code == kTileFull && (!cap || p.cap_raw) &&
-                (al == 0 || (al == 1 && __all_sync(0xffffffffu, !rvalid || A >= (float)(kPfCells - 1))));
+    const bool bits_tile = tiles.bits(kt);
+    bool fast = (code == kTileFull || bits_tile) && (!cap || p.cap_raw) &&
+                (al == 0 || (al == 1 && !tiles.late(kt)));
     if (fast) {
       uint32_t raw[kPfCells];
 #pragma unroll
@@ -627,7 +665,15 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       } else {
         tc_fence_before();
         mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
-        pf_weights<KT>(x, al == 1 ? C : 0.f, al == 1 ? 8.f * slope : 0.f, mt, m, l, mneg2, pk, need, factor);
+        const float boff = al == 1 ? C : 0.f, bstep = al == 1 ? 8.f * slope : 0.f;
+        if (bits_tile) {
+          const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
+                                        p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_t) << 2)))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+          vis[0] = bw.x; vis[1] = bw.y; vis[2] = bw.z; vis[3] = bw.w;
+          pf_apply_bits(x, vis, boff, bstep, mt);
+        }
+        pf_weights<KT>(x, boff, bstep, mt, m, l, mneg2, pk, need, factor);
       }
     }
     if (!fast) {

@@ -127,6 +127,32 @@ def test_deterministic(cuda_lib):
     a = run_prefill(p)
     b = run_prefill(p)
     assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    check(p, a, "bias + NaN V + ALiBi + softcap")
+
+
+def test_mask_bits_tiles(cuda_lib):
+    """A 0 / -inf causal mask with ALiBi, softcap and NaN V: the diagonal tiles
+    take the packed path with the classifier's visibility bits, and those
+    holding a NaN V run P V on the CUDA cores over the visible cells only."""
+    p = W.random_prefill(506, R=300, Hq=8, Hkv=2, D=128, depth=500, causal_by="mask", nan_v=4,
+                         alibi=True, sinks=True, softcap=40.0)
+    out = run_prefill(p)
+    ref = oracle.attn(p)
+    assert np.isnan(ref).any() and np.isfinite(ref).any()
+    check(p, out, "mask bits", ref=ref)
+
+
+@pytest.mark.parametrize("alibi", [False, True])
+def test_noncausal_zero_mask(cuda_lib, alibi):
+    """A 0 / -inf mask that lets rows see cells after their own position: with
+    ALiBi those tiles carry |row_pos - cell_pos| on both sides of the row."""
+    p = W.random_prefill(507, R=200, Hq=4, Hkv=1, D=128, depth=300, causal_by="mask", alibi=alibi,
+                         softcap=30.0)
+    rng = np.random.default_rng(7)
+    m = np.zeros(tuple(p.mask.shape), dtype=np.float32)
+    m[rng.random(m.shape) < 0.1] = -np.inf
+    p = dataclasses.replace(p, mask=torch.from_numpy(m))
+    check(p, run_prefill(p), f"non-causal mask alibi={alibi}")
 
 
 @pytest.fixture(scope="module")
