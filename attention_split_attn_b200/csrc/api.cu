@@ -368,6 +368,95 @@ PrefillWs prefill_ws_layout(const attn_args* a) {
   return w;
 }
 
+void record_event(void* const* events, int i, cudaStream_t s) {
+  if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+}
+
+// ---- unified-cache route (decode and prefill) -----------------------------------
+// With per-cell sequence ids the cells of a row's sequence are scattered over
+// the cache, so the dense kernels would stream every cell for every row.
+// Instead each row's visible cells are listed (same sequence, causal, mask
+// != -inf) and the selected-key gather kernel runs on the lists, adding the
+// mask bias per cell; rows are split into parts (folded by split_k_reduce)
+// as for the selected op.  Taken for 16-bit K/V with Q in their dtype, and
+// with ALiBi only when cell and row positions are given (the gather kernel's
+// distances use them as they are).
+bool unified_route(const attn_args* a) {
+  return a->cell_seq && a->row_seq && a->n_cells > 0 && (a->kv_type == ATTN_F16 || a->kv_type == ATTN_BF16) &&
+         a->q_type == a->kv_type && (reinterpret_cast<uintptr_t>(a->q) & 3u) == 0 && a->q_stride_row % 2 == 0 &&
+         a->q_stride_head % 2 == 0 && (!a->alibi_slopes || (a->cell_pos && a->row_pos));
+}
+
+// Parts per row: forced by n_slices, else enough that a part holds at most
+// about 4096 cells of the longest possible list (rows' lists differ wildly in
+// length; a part past the end of its row's list exits at once).
+SelShape plan_unified(const attn_args* a, int sms) {
+  if (a->n_slices > 0) return plan_selected(a, a->n_cells, sms);
+  const int64_t max_len = a->max_row_len > 0 ? std::min(a->max_row_len, a->n_cells) : a->n_cells;
+  const int64_t S = std::min<int64_t>(64, std::max<int64_t>(1, (max_len + 4095) / 4096));
+  SelShape sh;
+  sh.S = (int32_t)S;
+  int64_t C = (a->n_cells + S - 1) / S;
+  C = (C + 31) / 32 * 32;
+  sh.C = (int32_t)std::max<int64_t>(C, 32);
+  return sh;
+}
+
+size_t unified_ws_bytes(const attn_args* a, int sms) {
+  return selected_ws_layout(a, a->n_cells, plan_unified(a, sms)).total;
+}
+
+int32_t run_unified(const attn_args* a, void* ws, size_t ws_bytes, cudaStream_t s, void* const events[3],
+                    const DeviceInfo* di) {
+  const SelShape sh = plan_unified(a, di->sms);
+  const SelWs wl = selected_ws_layout(a, a->n_cells, sh);
+  if (ws == nullptr || ws_bytes < wl.total)
+    return fail(ATTN_ERR_WORKSPACE, "unified-cache attention needs %zu workspace bytes, got %zu", wl.total, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(ATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const int64_t blocks = (int64_t)a->n_rows * a->n_head_kv * sh.S;
+  if (blocks > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid of %lld CTAs is too large", (long long)blocks);
+  char* wsb = static_cast<char*>(ws);
+  SelectedPlan p{};
+  p.R = a->n_rows; p.Hq = a->n_head_q; p.Hkv = a->n_head_kv; p.G = a->n_head_q / a->n_head_kv;
+  p.D = a->head_dim; p.N = a->n_cells;
+  p.q = a->q; p.q_sr = a->q_stride_row; p.q_sh = a->q_stride_head;
+  p.k = a->k; p.v = a->v; p.kv_sc = a->kv_stride_cell; p.kv_sh = a->kv_stride_head; p.kv_type = a->kv_type;
+  p.out = OutSpec{a->out, a->out_type, a->o_stride_row, a->o_stride_head};
+  p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
+  p.cell_pos = a->cell_pos; p.row_pos = a->row_pos;
+  p.mask = a->mask; p.mask_sr = a->mask_stride_row;
+  p.n_sel = a->n_cells;   // row stride of the lists
+  p.compact = reinterpret_cast<int32_t*>(wsb);
+  p.count = reinterpret_cast<int32_t*>(wsb + wl.count_off);
+  p.S = sh.S; p.C = sh.C;
+  if (sh.S > 1) {
+    p.part.o = reinterpret_cast<float*>(wsb + wl.o_off);
+    p.part.ml = reinterpret_cast<float*>(wsb + wl.ml_off);
+    p.part.S = sh.S;
+  }
+  p.status = di->status;
+  const RowFilter f{a->row_begin, a->row_end, a->cell_seq, a->row_seq, a->cell_pos, a->row_pos,
+                    a->causal, a->mask, a->mask_stride_row};
+  record_event(events, 0, s);
+  cudaError_t e = launch_visible_lists(p, f, s);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "visible-list launch: %s", cudaGetErrorString(e));
+  e = launch_selected(p, s);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "gather launch: %s", cudaGetErrorString(e));
+  record_event(events, 1, s);
+  if (sh.S > 1) {
+    CombinePlan cp{};
+    cp.R = a->n_rows; cp.Hq = a->n_head_q; cp.Hkv = a->n_head_kv; cp.G = p.G; cp.D = a->head_dim;
+    cp.out = p.out; cp.sinks = a->sinks; cp.part = p.part;
+    cp.mode = 0;
+    cp.row_len = p.count; cp.C = sh.C; cp.N = a->n_cells;
+    cp.use_pdl = (events && events[1]) ? 0 : 1;
+    e = launch_combine(cp, s);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  }
+  record_event(events, 2, s);
+  return ATTN_OK;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -410,22 +499,15 @@ size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
   DeviceInfo* di = nullptr;
   if (device_info(&di) == ATTN_OK) sms = di->sms;
   switch (op) {
-    case ATTN_OP_DECODE: return decode_ws_bytes(a, plan_decode(a, sms));
+    case ATTN_OP_DECODE: return unified_route(a) ? unified_ws_bytes(a, sms) : decode_ws_bytes(a, plan_decode(a, sms));
     case ATTN_OP_SELECTED:
       if (n_sel < 1 || n_sel > kMaxSel) return 0;
       return selected_ws_layout(a, n_sel, plan_selected(a, n_sel, sms)).total;
-    case ATTN_OP_PREFILL: return prefill_ws_layout(a).total;
+    case ATTN_OP_PREFILL: return unified_route(a) ? unified_ws_bytes(a, sms) : prefill_ws_layout(a).total;
     default: return 0;
   }
 }
 
-namespace attn {
-namespace {
-void record_event(void* const* events, int i, cudaStream_t s) {
-  if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
-}
-}  // namespace
-}  // namespace attn
 
 int32_t attn_decode(const attn_args* a, void* ws, size_t ws_bytes, void* stream) {
   return attn_decode_timed(a, ws, ws_bytes, stream, nullptr);
@@ -438,6 +520,7 @@ int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* s
   if (a->n_rows == 0) return ATTN_OK;
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != ATTN_OK) return st;
+  if (unified_route(a)) return run_unified(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), events, di);
   const DecodeShape sh = plan_decode(a, di->sms);
   const size_t need = decode_ws_bytes(a, sh);
   if (need > 0 && (ws == nullptr || ws_bytes < need))
@@ -588,6 +671,7 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   if (a->n_rows == 0) return ATTN_OK;
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != ATTN_OK) return st;
+  if (unified_route(a)) return run_unified(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), events, di);
   const PrefillWs wl = prefill_ws_layout(a);
   if (wl.total > 0 && (ws == nullptr || ws_bytes < wl.total))
     return fail(ATTN_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", wl.total, ws_bytes);

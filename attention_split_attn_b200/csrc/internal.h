@@ -90,6 +90,8 @@ struct SelectedPlan {
   OutSpec out;
   Logits lg;
   const int32_t *cell_pos, *row_pos;   // ALiBi distances only
+  const float* mask;                   // optional F32 bias [R][mask_sr] added per listed cell
+  int64_t mask_sr;                     //   (unified-cache route; NULL for the selected op)
   const int32_t* sel;                  // [R][sel_stride], first n_sel used
   int64_t sel_stride;
   int32_t n_sel, n_pow2;               // n_pow2: n_sel rounded up to a power of 2
@@ -104,6 +106,13 @@ struct SelectedPlan {
 int selected_pow2(int n_sel);
 cudaError_t launch_select_compact(const SelectedPlan& p, cudaStream_t stream);
 cudaError_t launch_selected(const SelectedPlan& p, cudaStream_t stream);
+
+// Unified-cache route of decode and prefill (per-cell sequence ids): one CTA
+// per row scans the row's cell range and writes the visible cells (same
+// sequence, causal, mask != -inf) in ascending order into compact[r][0..),
+// their number into count[r]; the selected-key gather kernel then runs on
+// those lists with the mask bias added per cell.
+cudaError_t launch_visible_lists(const SelectedPlan& p, const RowFilter& f, cudaStream_t stream);
 
 // ---- causal prefill -----------------------------------------------------------
 // Tiles of 128 query rows x 128 cells.  A classifier kernel tags every (row

@@ -209,7 +209,8 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <typename KT, int D, int NH>
+// BIAS: add the F32 mask bias of each listed cell (unified-cache route only).
+template <typename KT, int D, int NH, bool BIAS>
 __global__ void __launch_bounds__(SelCfg<KT, D, NH>::THREADS)
 selected_kernel(const SelectedPlan p) {
   using C = SelCfg<KT, D, NH>;
@@ -388,11 +389,14 @@ selected_kernel(const SelectedPlan p) {
         const int idx = tile0 + mt * 16 + grp + 8 * kr;
         const bool vk = idx < c_end;
         vis[mt][kr] = vk;
-        float negdist = 0.f;
-        if (alibi && vk) {
+        float negdist = 0.f, bias = 0.f;
+        if ((alibi || BIAS) && vk) {
           const int c = __ldg(cells + idx);
-          const int64_t cpos = p.cell_pos ? (int64_t)__ldg(p.cell_pos + c) : (int64_t)c;
-          negdist = -(float)(row_pos >= cpos ? row_pos - cpos : cpos - row_pos);
+          if (alibi) {
+            const int64_t cpos = p.cell_pos ? (int64_t)__ldg(p.cell_pos + c) : (int64_t)c;
+            negdist = -(float)(row_pos >= cpos ? row_pos - cpos : cpos - row_pos);
+          }
+          if (BIAS) bias = __ldg(p.mask + (int64_t)r * p.mask_sr + c);   // F32, added unnarrowed
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -401,6 +405,7 @@ selected_kernel(const SelectedPlan p) {
             float x = sc[mt][nt][2 * kr + e] * scale;
             if (softcap > 0.f) x = softcap * tanhf(x / softcap);
             if (alibi) x = fmaf(slope[nt][e], negdist, x);
+            if (BIAS) x += bias;
             sc[mt][nt][2 * kr + e] = vk ? x : neg_inf();
           }
       }
@@ -530,13 +535,74 @@ selected_kernel(const SelectedPlan p) {
 template <typename KT, int D, int NH>
 cudaError_t launch_selected_t(const SelectedPlan& p, cudaStream_t stream) {
   using C = SelCfg<KT, D, NH>;
-  auto kern = selected_kernel<KT, D, NH>;
-  static std::atomic<unsigned long long> smem_set{0ull};
-  cudaError_t e = set_smem_limit_once(smem_set, kern, C::TOTAL);
+  auto kern = p.mask ? selected_kernel<KT, D, NH, true> : selected_kernel<KT, D, NH, false>;
+  static std::atomic<unsigned long long> smem_set{0ull}, smem_set_b{0ull};
+  cudaError_t e = set_smem_limit_once(p.mask ? smem_set_b : smem_set, kern, C::TOTAL);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)p.R * p.Hkv * p.S;
   kern<<<dim3((unsigned)blocks), C::THREADS, C::TOTAL, stream>>>(p);
   return cudaGetLastError();
+}
+
+// ---- unified-cache route: the visible cells of each row, in order ------------
+// One CTA of 1024 threads per row.  Each round covers 4096 cells as four
+// 1024-cell sub-chunks: the loads of all four go out first, then each
+// sub-chunk is compacted in order (warp ballots, a prefix over the 32 warp
+// counts in shared memory).
+constexpr int kVisThreads = 1024;
+
+__global__ void __launch_bounds__(kVisThreads) visible_list_kernel(const SelectedPlan p, const RowFilter f) {
+  __shared__ int wcount[32];
+  __shared__ int base_sh;
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  int32_t rb = f.row_begin ? __ldg(f.row_begin + r) : 0;
+  int32_t re = f.row_end ? __ldg(f.row_end + r) : p.N;
+  rb = max(rb, 0);
+  re = min(re, p.N);
+  const int32_t rs = f.row_seq ? __ldg(f.row_seq + r) : 0;
+  const int32_t rp = f.row_pos ? __ldg(f.row_pos + r) : re - rb - 1;
+  const float* mrow = f.mask ? f.mask + (int64_t)r * f.mask_sr : nullptr;
+  int32_t* out = p.compact + (int64_t)r * p.n_sel;
+  if (tid == 0) base_sh = 0;
+  __syncthreads();
+  for (int64_t c0 = rb; c0 < re; c0 += 4 * kVisThreads) {
+    bool vis[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t c = c0 + k * kVisThreads + tid;
+      bool v = c < re;
+      if (v && f.cell_seq) v = __ldg(f.cell_seq + c) == rs;
+      if (v && f.causal) {
+        const int32_t cp = f.cell_pos ? __ldg(f.cell_pos + c) : (int32_t)(c - rb);
+        v = cp <= rp;
+      }
+      if (v && mrow) v = !(__ldg(mrow + c) == neg_inf());
+      vis[k] = v;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const unsigned bal = __ballot_sync(0xffffffffu, vis[k]);
+      if (lane == 0) wcount[wid] = __popc(bal);
+      __syncthreads();
+      if (wid == 0) {
+        const int x = wcount[lane];
+        int incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        wcount[lane] = incl - x;   // exclusive prefix of the warp counts
+      }
+      __syncthreads();
+      const int base = base_sh;
+      if (vis[k]) out[base + wcount[wid] + __popc(bal & ((1u << lane) - 1u))] = (int32_t)(c0 + k * kVisThreads + tid);
+      __syncthreads();
+      if (tid == kVisThreads - 1) base_sh = base + wcount[31] + __popc(bal);
+      __syncthreads();
+    }
+  }
+  if (tid == 0) p.count[r] = base_sh;
 }
 
 template <typename KT>
@@ -570,6 +636,11 @@ cudaError_t launch_select_compact(const SelectedPlan& p, cudaStream_t stream) {
   // at most 4096 keys + the scan scratch: 16.5 KB, under the default limit
   const size_t smem = ((size_t)p.n_pow2 + kSortThreads / 32) * sizeof(int32_t);
   select_compact_kernel<<<dim3((unsigned)p.R), kSortThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_visible_lists(const SelectedPlan& p, const RowFilter& f, cudaStream_t stream) {
+  visible_list_kernel<<<dim3((unsigned)p.R), kVisThreads, 0, stream>>>(p, f);
   return cudaGetLastError();
 }
 

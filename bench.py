@@ -20,7 +20,9 @@ workloads, per call with the L2 flushed before each call: maskless
 selected-key attention (2048 rows, GQA 12, D 256, fp16 cache of 32768 cells;
 effective GB/s of the gathered K/V rows) and causal prefill (2048 rows over
 14048 cells, Hq 64 / Hkv 8, D 128, bf16; TFLOP/s over the visible pairs on
-the tensor cores), each with the roofline of its main kernel.
+the tensor cores), and the unified-cache semantics sweep through attn_decode and
+attn_prefill (GB/s of the visible K/V rows, mask rows and cell metadata), each
+with the roofline of its main kernel.
 --profile-op {decode,selected,prefill} only runs W + K calls of one operation
 (the command the ncu summaries under profiles/ are taken on).
 
@@ -413,7 +415,49 @@ def run_parts(args, rank, dev, stream):
                      "kernel_ms": main, "algorithmic_flops": flops,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS)"},
     }
+    del q, k, v, out, pa, ws, kw
+
+    # semantics sweep: unified fp16 cache of 8 interleaved sequences, 256 rows,
+    # per-cell sequence ids and positions, F32 mask, NaN cells, sinks; through
+    # attn_decode (planner slices) and attn_prefill.  Bytes: the K and V rows of
+    # every visible (cell, KV head), the F32 mask rows and the cell metadata
+    # each row scans, Q and the output.
+    p = W.semantics_sweep()
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    vis = _visible_cells(p)
+    nbytes = (vis * p.n_head_kv * p.head_dim * p.k.element_size() * 2
+              + p.n_rows * p.n_cells * (4 + 8) + p.q.numel() * p.q.element_size()
+              + p.n_rows * p.n_head_q * p.head_dim * 4)
+    for name, op, call in (("semantics_decode", A.OP_DECODE, A.attn_decode_timed_args),
+                           ("semantics_prefill", A.OP_PREFILL, A.attn_prefill_timed_args)):
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, op), 256), dtype=torch.uint8, device=dev)
+        for _ in range(max(args.warmup, 3)):
+            (A.attn_decode_args if op == A.OP_DECODE else A.attn_prefill_args)(a, ws=ws, stream=stream)
+        whole, main = _time_calls(lambda e: call(a, ws, e, stream=stream), n, flush, stream)
+        parts[name] = {
+            "workload": "semantics_sweep: unified fp16 cache of 8 interleaved sequences, 256 rows with lengths "
+                        "log-uniform in [1, 65536], Hq 16 / Hkv 4, D 128, F32 mask with -inf/+inf, NaN cells, sinks",
+            "value": nbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (visible K/V + mask + cell metadata)",
+            "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
+            "gpu_launches": (2 if op == A.OP_PREFILL else 3) * n,
+            "roofline": {"bound": "hbm", "achieved": nbytes / (main * 1e-3) / 1e9, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None,
+                         "kernel_ms": main, "algorithmic_bytes": nbytes,
+                         "peak_kind": f"{peak_kind} hbm_gbs (burst copy); semantics case, no target"},
+        }
     return parts
+
+
+def _visible_cells(p) -> int:
+    """Number of visible (row, cell) pairs: same sequence, causal, mask not -inf."""
+    cs, cp = p.cell_seq.numpy(), p.cell_pos.numpy()
+    rs, rp = p.row_seq.numpy(), p.row_pos.numpy()
+    m = p.mask.numpy()
+    total = 0
+    for r in range(p.n_rows):
+        total += int(((cs == rs[r]) & (cp <= rp[r]) & (m[r] != -np.inf)).sum())
+    return total
 
 
 def run_profile_op(args, local):
