@@ -30,6 +30,15 @@
  *                  and grid_order are ignored.  Workspace: one byte per
  *                  (128-row tile, 128-cell tile) and per (cell tile, KV head).
  *
+ * Unified caches.  When cell_seq/row_seq are given (several sequences'
+ * cells interleaved in one cache, strix-llama.cpp PR #115 "Isolation"), the
+ * cells a row may see are scattered, so attn_decode and attn_prefill first
+ * list each row's visible cells (ascending) and then gather them in blocks
+ * of 32 cells as attn_selected does, adding the F32 mask bias per cell; rows
+ * are split into parts folded by split_k_reduce.  This route needs F16/BF16
+ * K/V with Q in that dtype (and cell_pos/row_pos when ALiBi slopes are
+ * given); its workspace holds one int32 list of n_cells entries per row.
+ *
  * Semantics (all three; HartsyInference PR #910 "attention semantic
  * correctness"):  for row r and query head h (KV head g = h / (Hq/Hkv)),
  *   x_c = scale * q.k_c;  x_c = softcap*tanh(x_c/softcap) if softcap > 0;
