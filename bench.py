@@ -23,7 +23,7 @@ effective GB/s of the gathered K/V rows) and causal prefill (2048 rows over
 the tensor cores), and the unified-cache semantics sweep through attn_decode and
 attn_prefill (GB/s of the visible K/V rows, mask rows and cell metadata), each
 with the roofline of its main kernel.
---profile-op {decode,selected,prefill} only runs W + K calls of one operation
+--profile-op {decode,selected,prefill,semantics} only runs W + K calls of one operation
 (the command the ncu summaries under profiles/ are taken on).
 
 --impl reference times the FP64 CPU oracle on the host cores on a bounded
@@ -383,7 +383,8 @@ def run_parts(args, rank, dev, stream):
                     "2048-entry lists (5% dup, 3% invalid), f32 out",
         "value": nbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (effective: gathered K/V bytes)",
         "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
-        "gpu_launches": 3 * n,
+        # compaction + gather (2048 rows x 4 KV heads fill the GPU: one part per row, no combine)
+        "gpu_launches": 2 * n,
         "roofline": {"bound": "hbm", "achieved": nbytes / (main * 1e-3) / 1e9, "peak": hbm_peak,
                      "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak,
                      "traffic": _recorded_traffic("selected_kernel"),
@@ -440,7 +441,8 @@ def run_parts(args, rank, dev, stream):
                         "log-uniform in [1, 65536], Hq 16 / Hkv 4, D 128, F32 mask with -inf/+inf, NaN cells, sinks",
             "value": nbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (visible K/V + mask + cell metadata)",
             "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
-            "gpu_launches": (2 if op == A.OP_PREFILL else 3) * n,
+            # visible lists + gather + split_k_reduce (long rows are split into parts)
+            "gpu_launches": 3 * n,
             "roofline": {"bound": "hbm", "achieved": nbytes / (main * 1e-3) / 1e9, "peak": hbm_peak,
                          "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None,
                          "kernel_ms": main, "algorithmic_bytes": nbytes,
@@ -469,6 +471,12 @@ def run_profile_op(args, local):
     op = args.profile_op
     if op == "decode":
         p = W.gqa_decode(poison_unused=False)
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_decode_args(a, ws=ws)
+    elif op == "semantics":
+        p = W.semantics_sweep()
         (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
         a = A.make_args(q, k, v, out, **kw)
         ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
@@ -543,7 +551,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-parts", action="store_true", help="time the decode workload only")
-    ap.add_argument("--profile-op", choices=["decode", "selected", "prefill"], default=None,
+    ap.add_argument("--profile-op", choices=["decode", "selected", "prefill", "semantics"], default=None,
                     help="only run W + K calls of one operation (for ncu captures); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
