@@ -565,6 +565,7 @@ int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* s
   if (sh.stream) {
     p.W = sh.W;
     p.row_tiles = reinterpret_cast<int64_t*>(wsb + wl.tiles_off);
+    p.plan_inline = a->n_rows <= 64 ? 1 : 0;   // kInlineRows of the stream kernel
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   record_event(events, 0, s);

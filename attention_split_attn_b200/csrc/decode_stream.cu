@@ -21,7 +21,8 @@
 //
 // A planner kernel first writes row_tiles[r] (exclusive prefix of each row's
 // tile count); the persistent kernel and the combine run behind it with
-// programmatic dependent launch.
+// programmatic dependent launch.  With at most kInlineRows rows every warp
+// computes the prefix itself and no planner runs.
 #include "common.cuh"
 #include "decode_tile.cuh"
 #include "internal.h"
@@ -31,11 +32,16 @@ namespace attn {
 
 namespace {
 
+// Up to this many rows, every warp computes the row tile prefix itself (no
+// planner kernel in front of the stream kernel).
+constexpr int kInlineRows = 64;
+
 template <int D>
 struct StreamRing {
   static constexpr int NS = 2;                       // ring stages per warp
   static constexpr int BAR_OFF = NS * WarpStage<D>::BYTES;
-  static constexpr int TOTAL = BAR_OFF + NS * 8 + 1024;   // + alignment slack for the swizzle
+  static constexpr int RT_OFF = BAR_OFF + NS * 8;    // inline row tile prefix [kInlineRows + 1]
+  static constexpr int TOTAL = RT_OFF + (kInlineRows + 1) * 8 + 1024;   // + alignment slack for the swizzle
 };
 
 __device__ __forceinline__ int64_t row_len(const DecodePlan& p, int r) {
@@ -88,8 +94,8 @@ struct Cursor {
   int32_t begin, end;
 };
 
-__device__ __forceinline__ void cursor_load_row(const DecodePlan& p, Cursor& c) {
-  c.nt = p.row_tiles[c.r + 1] - p.row_tiles[c.r];
+__device__ __forceinline__ void cursor_load_row(const DecodePlan& p, const int64_t* row_tiles, Cursor& c) {
+  c.nt = row_tiles[c.r + 1] - row_tiles[c.r];
   int32_t b = p.f.row_begin ? __ldg(p.f.row_begin + c.r) : 0;
   int32_t e = p.f.row_end ? __ldg(p.f.row_end + c.r) : p.N;
   b = max(b, 0);
@@ -99,14 +105,14 @@ __device__ __forceinline__ void cursor_load_row(const DecodePlan& p, Cursor& c) 
 }
 
 // Move to the next tile; rows without tiles are skipped.
-__device__ __forceinline__ void cursor_next(const DecodePlan& p, Cursor& c) {
+__device__ __forceinline__ void cursor_next(const DecodePlan& p, const int64_t* row_tiles, Cursor& c) {
   if (++c.j < c.nt) return;
   c.j = 0;
   if (++c.g < p.Hkv) return;
   c.g = 0;
   do {
     ++c.r;
-    cursor_load_row(p, c);
+    cursor_load_row(p, row_tiles, c);
   } while (c.nt == 0 && c.r + 1 < p.R);
 }
 
@@ -125,10 +131,37 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   }
   __syncwarp();
   pdl_launch_dependents();
-  pdl_wait_prior_grid();   // row_tiles from the planner
+  // The row tile prefix: from the planner, or (few rows) computed here
+  // before waiting on the previous kernel in the stream, which may still be
+  // reading a workspace this call is about to reuse.
+  const int64_t* row_tiles = p.row_tiles;
+  if (p.plan_inline) {
+    int64_t* rt = reinterpret_cast<int64_t*>(smem + StreamRing<D>::RT_OFF);
+    int64_t carry = 0;
+    for (int base = 0; base < p.R; base += 32) {
+      const int r = base + lane;
+      const int64_t n = r < p.R ? (row_len(p, r) + kWarpTile - 1) / kWarpTile : 0;
+      int64_t x = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+      }
+      if (r < p.R) rt[r] = carry + x - n;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) rt[p.R] = carry;
+    __syncwarp();
+    row_tiles = rt;
+  }
+  pdl_wait_prior_grid();
+  if (p.plan_inline && blockIdx.x == 0) {
+    // the combine reads the prefix from the workspace
+    for (int r = lane; r <= p.R; r += 32) p.row_tiles[r] = row_tiles[r];
+  }
 
   const int64_t W = p.W, Hkv = p.Hkv;
-  const int64_t T = Hkv * p.row_tiles[p.R];
+  const int64_t T = Hkv * row_tiles[p.R];
   const int64_t w = p.grid_order ? W - 1 - blockIdx.x : blockIdx.x;
   const int64_t t0 = T * w / W, t1 = T * (w + 1) / W;
   if (t0 >= t1) return;
@@ -140,7 +173,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     const int64_t span = hi - lo;
     const int64_t step = (span + 31) / 32;
     const int64_t probe = lo + lane * step;
-    const bool ok = probe < hi && Hkv * p.row_tiles[probe] <= t0;
+    const bool ok = probe < hi && Hkv * row_tiles[probe] <= t0;
     const unsigned m = __ballot_sync(0xffffffffu, ok);
     const int k = 31 - __clz(m);       // lane 0 always qualifies (row_tiles[lo] <= t0)
     lo = (int)(lo + k * step);
@@ -148,9 +181,9 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   }
   Cursor c;
   c.r = lo;
-  cursor_load_row(p, c);
+  cursor_load_row(p, row_tiles, c);
   {
-    const int64_t off = t0 - Hkv * p.row_tiles[c.r];
+    const int64_t off = t0 - Hkv * row_tiles[c.r];
     c.g = (int)(off / c.nt);
     c.j = off % c.nt;
   }
@@ -163,7 +196,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   if (lane == 0) {
     pol = policy_evict_first();
     for (; issued < (n < NS ? n : (int64_t)NS); ++issued) {
-      if (issued > 0) cursor_next(p, ic);
+      if (issued > 0) cursor_next(p, row_tiles, ic);
       issue_warp_tile<D>(smem + issued * WarpStage<D>::BYTES, &full[issued], &tmK, &tmV, ic.g,
                          ic.begin + (int)(ic.j * kWarpTile), pol);
     }
@@ -201,7 +234,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       if (lane == 0 && issued < n) {
         // the lanes' shared-memory reads of this stage precede its async refill
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        cursor_next(p, ic);
+        cursor_next(p, row_tiles, ic);
         issue_warp_tile<D>(stage, &full[stg], &tmK, &tmV, ic.g, ic.begin + (int)(ic.j * kWarpTile), pol);
         ++issued;
       }
@@ -214,11 +247,11 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       // the pair ends here (or this warp's run does): emit its record
       st.finish_sums();
       const int64_t pair = (int64_t)c.r * Hkv + c.g;
-      const int64_t pair_start = Hkv * p.row_tiles[c.r] + (int64_t)c.g * c.nt;
+      const int64_t pair_start = Hkv * row_tiles[c.r] + (int64_t)c.g * c.nt;
       const int64_t slot = pair_start >= t0 ? W + pair : w;
       st.write_partial(p.part.o, p.part.ml, slot, p.G, lane, false);
       if (!last) {
-        cursor_next(p, c);
+        cursor_next(p, row_tiles, c);
         rc = make_ctx(c);
         st.reset();
         st.load_q(p, c.r, c.g * p.G, lane);
@@ -230,7 +263,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   if (aborted) {
     // poison the record in progress and leave no copy in flight
     const int64_t pair = (int64_t)c.r * Hkv + c.g;
-    const int64_t pair_start = Hkv * p.row_tiles[c.r] + (int64_t)c.g * c.nt;
+    const int64_t pair_start = Hkv * row_tiles[c.r] + (int64_t)c.g * c.nt;
     st.write_partial(p.part.o, p.part.ml, pair_start >= t0 ? W + pair : w, p.G, lane, true);
     if (lane == 0)
       for (int64_t kk = k; kk < issued; ++kk) mbar_wait_bounded(&full[kk % NS], (uint32_t)((kk / NS) & 1), nullptr);
@@ -245,8 +278,10 @@ cudaError_t launch_stream_t(const DecodePlan& p, const CUtensorMap& tmK, const C
   static std::atomic<unsigned long long> smem_set{0ull};
   cudaError_t e = set_smem_limit_once(smem_set, kern, StreamRing<D>::TOTAL);
   if (e != cudaSuccess) return e;
-  decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!p.plan_inline) {
+    decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.W);
   cfg.blockDim = dim3(32);

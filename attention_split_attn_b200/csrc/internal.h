@@ -64,6 +64,7 @@ struct DecodePlan {
   // balanced persistent scheme (n_slices == 0 with the tensor-core kernels):
   int32_t W;          // warps of the persistent grid
   int64_t* row_tiles; // [R+1] exclusive prefix of 16-cell tiles per row (planner output)
+  int32_t plan_inline; // 1: few rows; the stream kernel computes the prefix (no planner)
 };
 
 bool decode_uses_mma(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh);

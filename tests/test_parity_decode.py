@@ -17,7 +17,7 @@ import torch
 import oracle
 import attention_split_attn_b200 as A
 from attention_split_attn_b200 import workloads as W
-from parity import check, run_decode, tolerance, compare
+from parity import check, run_decode, tolerance, compare, poisoned_workspace
 
 pytestmark = pytest.mark.gpu
 
@@ -207,3 +207,24 @@ def test_balanced_more_warps_than_tiles(cuda_lib):
     p = W.random_problem(79, R=70, Hq=16, Hkv=1, D=256, N=300, kv_dtype=torch.bfloat16,
                          out_dtype=torch.float32, softcap=3.0)
     check(p, run_decode(p, n_slices=0), "many short rows")
+
+
+@pytest.mark.parametrize("R", [63, 64, 65, 200])
+def test_balanced_row_counts_around_inline_prefix(cuda_lib, R):
+    """Up to 64 rows every warp computes the row tile prefix itself; above
+    that a planner kernel does.  Both, with empty rows among them, and the
+    second call on the same workspace, give the oracle's result."""
+    rng = np.random.default_rng(R)
+    lengths = [int(x) for x in rng.integers(0, 700, size=R)]
+    lengths[R // 2] = 0
+    p = W.random_problem(900 + R, R=R, Hq=8, Hkv=2, D=128, N=800, kv_dtype=torch.bfloat16,
+                         out_dtype=torch.float32, lengths=lengths, sinks=True, causal=True)
+    ref = oracle.attn(p)
+    (q, k, v, out), kw = A.problem_kwargs(p)
+    args = A.make_args(q, k, v, out, **kw)
+    ws = poisoned_workspace(A.workspace_size(args, A.OP_DECODE))
+    for _ in range(2):
+        out.fill_(float("nan"))
+        A.attn_decode_args(args, ws=ws)
+        torch.cuda.synchronize()
+        check(p, out, f"R={R}", ref=ref)
