@@ -32,7 +32,7 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
            "attn_prefill", "attn_decode_timed", "attn_selected_timed", "attn_prefill_timed",
-           "attn_decode_noalloc",
+           "attn_decode_noalloc", "attn_tree_mask",
            "attn_check_device_status",
            "attn_strerror", "attn_last_error", "attn_abi_version")
 
@@ -109,6 +109,9 @@ def load_library():
             lib.attn_selected_timed.restype = ctypes.c_int32
             lib.attn_selected_timed.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
                                                 ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p * 3]
+            lib.attn_tree_mask.restype = ctypes.c_int32
+            lib.attn_tree_mask.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
             lib.attn_check_device_status.restype = ctypes.c_int32
             lib.attn_check_device_status.argtypes = [ctypes.c_void_p]
             lib.attn_strerror.restype = ctypes.c_char_p
@@ -319,6 +322,23 @@ def selected_workspace_size(args: AttnSelectedArgs) -> int:
 def selected(q, k, v, out, sel, *, ws=None, stream=None, **kw):
     """Maskless selected-key attention into `out` (see include/attn.h)."""
     return attn_selected_args(make_selected_args(q, k, v, out, sel, **kw), ws=ws, stream=stream)
+
+
+def tree_mask(parent: torch.Tensor, prefix_cells: int, n_cells: int, mask: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """The F32 mask [rows, n_cells] under which attn_decode computes draft-tree
+    rows: row r is node r (token in cell prefix_cells + r, parent parent[r] <
+    r or -1) and sees the prefix and its ancestors' cells (see include/attn.h)."""
+    _check_i32("parent", parent, parent.numel())
+    R = parent.numel()
+    if mask is None:
+        mask = torch.empty((R, n_cells), dtype=torch.float32, device=parent.device)
+    if mask.dtype != torch.float32 or mask.stride(1) != 1 or tuple(mask.shape) != (R, n_cells):
+        raise ValueError("mask must be float32 [rows, n_cells] with contiguous cells")
+    lib = load_library()
+    _raise_if(lib.attn_tree_mask(parent.data_ptr(), R, int(prefix_cells), int(n_cells), mask.data_ptr(),
+                                 mask.stride(0), _stream_handle(stream)), "attn_tree_mask")
+    return mask
 
 
 def check_device_status(stream=None):

@@ -756,6 +756,24 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   return ATTN_OK;
 }
 
+int32_t attn_tree_mask(const int32_t* parent, int32_t n_rows, int32_t prefix_cells, int32_t n_cells, float* mask,
+                       int64_t mask_stride_row, void* stream) {
+  if (n_rows < 0 || prefix_cells < 0 || n_cells < 0) return fail(ATTN_ERR_INVALID_ARG, "negative size");
+  if (n_rows == 0) return ATTN_OK;
+  if (!parent || !mask) return fail(ATTN_ERR_INVALID_ARG, "parent or mask is NULL");
+  if (n_rows > max_tree_rows()) return fail(ATTN_ERR_UNSUPPORTED, "tree of %d rows > %d", n_rows, max_tree_rows());
+  if (mask_stride_row < n_cells) return fail(ATTN_ERR_INVALID_ARG, "mask_stride_row is smaller than n_cells");
+  if ((int64_t)prefix_cells + n_rows > n_cells)
+    return fail(ATTN_ERR_INVALID_ARG, "the tree cells [prefix_cells, prefix_cells + n_rows) pass n_cells");
+  DeviceInfo* di = nullptr;
+  int32_t st = device_info(&di);
+  if (st != ATTN_OK) return st;
+  const cudaError_t e = launch_tree_mask(parent, n_rows, prefix_cells, n_cells, mask, mask_stride_row, di->status,
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "tree mask launch: %s", cudaGetErrorString(e));
+  return ATTN_OK;
+}
+
 int32_t attn_check_device_status(void* stream) {
   DeviceInfo* di = nullptr;
   int32_t st = device_info(&di);

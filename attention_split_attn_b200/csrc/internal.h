@@ -183,6 +183,11 @@ struct CombinePlan {
 };
 cudaError_t launch_combine(const CombinePlan& p, cudaStream_t stream);
 
+// ---- draft-tree rows ------------------------------------------------------------
+cudaError_t launch_tree_mask(const int32_t* parent, int32_t n_rows, int32_t prefix_cells, int32_t n_cells,
+                             float* mask, int64_t mask_sr, int* status, cudaStream_t stream);
+int max_tree_rows();
+
 // Set the message attn_last_error() returns on this thread.
 void set_last_error(const char* msg);
 

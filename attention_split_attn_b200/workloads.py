@@ -249,6 +249,35 @@ def semantics_sweep(seed: int = 1005, R: int = 256, n_seq: int = 8, max_len: int
                    sinks=torch.from_numpy(sinks), max_row_len=N)
 
 
+def tree_decode(seed: int = 1006, width: int = 16, visible: int = 32770, Hq: int = 32, Hkv: int = 8,
+                D: int = 128) -> Problem:
+    """Draft-tree decode rows (TensorFold PR #2595: tree table with heap-order
+    parents, widths 1..16, visible keys such as 33, 34, 8193, 32768..32770):
+    `width` rows, node i's parent (i - 1) // 2 (a binary heap; -1 for the
+    root), node i's token in cell prefix + i with prefix = visible - 1, so the
+    root sees `visible` cells.  Bf16 Q/K/V ~ N(0, 1), bf16 out.  The visibility
+    mask (0 for the prefix and the row's ancestors-or-self, -inf elsewhere) is
+    built here on the host for the oracle; the CUDA path builds its own."""
+    rng = np.random.default_rng(seed)
+    prefix = visible - 1
+    N = prefix + width
+    q = _normal(rng, (width, Hq, D), BF16)
+    k = _normal(rng, (N, Hkv, D), BF16)
+    v = _normal(rng, (N, Hkv, D), BF16)
+    parent = np.array([-1] + [(i - 1) // 2 for i in range(1, width)], dtype=np.int64)
+    mask = np.full((width, N), -np.inf, dtype=np.float32)
+    mask[:, :prefix] = 0.0
+    for r in range(width):
+        node = r
+        while node >= 0:
+            mask[r, prefix + node] = 0.0
+            node = parent[node]
+    p = Problem("tree_decode", q, k, v, out_dtype=BF16, scale=1.0 / math.sqrt(D), mask=torch.from_numpy(mask))
+    p.tree_parent = _i32(parent)
+    p.tree_prefix = prefix
+    return p
+
+
 WORKLOADS = {
     "tiny_decode": tiny_decode,
     "gqa_decode": gqa_decode,

@@ -20,9 +20,10 @@ workloads, per call with the L2 flushed before each call: maskless
 selected-key attention (2048 rows, GQA 12, D 256, fp16 cache of 32768 cells;
 effective GB/s of the gathered K/V rows) and causal prefill (2048 rows over
 14048 cells, Hq 64 / Hkv 8, D 128, bf16; TFLOP/s over the visible pairs on
-the tensor cores), and the unified-cache semantics sweep through attn_decode and
-attn_prefill (GB/s of the visible K/V rows, mask rows and cell metadata), each
-with the roofline of its main kernel.
+the tensor cores), draft-tree decode rows (tree mask + attn_decode), and the
+unified-cache semantics sweep through attn_decode and attn_prefill (GB/s of the
+visible K/V rows, mask rows and cell metadata), each with the roofline of its
+main kernel.
 --profile-op {decode,selected,prefill,semantics} only runs W + K calls of one operation
 (the command the ncu summaries under profiles/ are taken on).
 
@@ -417,6 +418,48 @@ def run_parts(args, rank, dev, stream):
                      "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS)"},
     }
     del q, k, v, out, pa, ws, kw
+
+    # draft-tree decode rows: 16 nodes of a binary draft tree over 130856 keys
+    # (the depth of TensorFold PR #2595's long-context receipt), GQA heads;
+    # a call = the tree mask kernel + attn_decode.  Algorithmic bytes: the K/V
+    # rows of every cell some row sees, once (the rows share the prefix), the
+    # mask, Q and the output; rows_per_s and the per-row view are beside it.
+    p = W.tree_decode(width=16, visible=130856)
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    kw.pop("mask")
+    parent = p.tree_parent.to(dev)
+    tmask = torch.empty((p.n_rows, p.n_cells), dtype=torch.float32, device=dev)
+    ta = A.make_args(q, k, v, out, mask=tmask, **kw)
+    ws = torch.empty(max(A.workspace_size(ta, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+    vis = int(torch.isfinite(p.mask).sum())
+    cells = int(torch.isfinite(p.mask).any(dim=0).sum())
+    kv_cell = p.n_head_kv * p.head_dim * p.k.element_size() * 2
+    rest = p.n_rows * p.n_cells * 4 + p.q.numel() * p.q.element_size() + p.n_rows * p.n_head_q * p.head_dim * 2
+    tbytes = cells * kv_cell + rest
+
+    def tree_call(e):
+        e[0].record(stream)
+        A.tree_mask(parent, p.tree_prefix, p.n_cells, mask=tmask, stream=stream)
+        A.attn_decode_args(ta, ws=ws, stream=stream)
+        e[1].record(stream)
+        e[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        tree_call([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    whole, main = _time_calls(tree_call, n, flush, stream)
+    parts["tree_decode"] = {
+        "workload": "tree_decode: 16 draft-tree rows (binary heap order) over 130856 keys, Hq 32 / Hkv 8, D 128, "
+                    "bf16 KV and out; tree mask + attn_decode",
+        "value": tbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (K/V of every visible cell once + mask)",
+        "per_row_GBs": (vis * kv_cell + rest) / (whole * 1e-3) / 1e9,
+        "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
+        "gpu_launches": 3 * n,   # tree mask + stream kernel + split_k_reduce
+        "roofline": {"bound": "hbm", "achieved": tbytes / (main * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": tbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None, "kernel_ms": main,
+                     "algorithmic_bytes": tbytes,
+                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy); each row streams the shared prefix"},
+    }
+    del q, k, v, out, ta, ws, kw, tmask
 
     # semantics sweep: unified fp16 cache of 8 interleaved sequences, 256 rows,
     # per-cell sequence ids and positions, F32 mask, NaN cells, sinks; through

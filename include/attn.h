@@ -198,6 +198,20 @@ int32_t attn_prefill_timed(const attn_args *args, void *ws, size_t ws_bytes, voi
  *    (cudaGetSymbolAddress, no allocation); make it before any stream capture. */
 int32_t attn_decode_noalloc(const attn_args *args, void *stream);
 
+/* Draft-tree rows (TensorFold PR #2595: attn_decode over "Q rows, K/V cache,
+ * tree table" with heap-order parents, tree widths 1..16).  Writes the F32
+ * additive mask [n_rows][n_cells] (row stride mask_stride_row, DEVICE memory)
+ * under which attn_decode computes the tree rows: row r is tree node r, whose
+ * token is in cell prefix_cells + r; parent[r] (DEVICE, int32) is its parent
+ * node, smaller than r, or -1 for a root.  Row r sees cells [0, prefix_cells)
+ * and the cells of its ancestors and itself (mask 0); every other cell is
+ * -inf.  n_rows <= 4096; prefix_cells + n_rows <= n_cells.  A parent that is
+ * not smaller than its child records ATTN_ERR_INVALID_ARG in the device status
+ * word (attn_check_device_status) and hides the ancestors above it.
+ * Asynchronous on `stream`; allocates nothing.                              */
+int32_t attn_tree_mask(const int32_t *parent, int32_t n_rows, int32_t prefix_cells, int32_t n_cells,
+                       float *mask, int64_t mask_stride_row, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word on the
  * current device: ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on
  * a bounded wait since the last check.                                      */

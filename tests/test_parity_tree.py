@@ -1,0 +1,84 @@
+"""Draft-tree decode rows on a B200 (attn_tree_mask + attn_decode).
+
+TensorFold PR #2595 decodes the nodes of a draft tree as the rows of one
+attn_decode call (tree table with heap-order parents; its kernel contract
+checks tree widths 1, 2, 4, 8, 12, 16 at 33, 34, 8193, 32768, 32769 and 32770
+visible keys).  Here the visibility mask comes from the library's tree-mask
+kernel; it must equal the mask the workload generator builds on the host, and
+the decoded rows must match the FP64 oracle under the host mask.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import attention_split_attn_b200 as A
+from attention_split_attn_b200 import workloads as W
+from parity import check, poisoned_workspace
+
+pytestmark = pytest.mark.gpu
+
+WIDTHS = [1, 2, 4, 8, 12, 16]
+KEYS = [33, 34, 8193, 32768, 32769, 32770]
+
+
+def decode_tree(p, n_slices=0, grid_order=0):
+    (q, k, v, out), kw = A.problem_kwargs(p)
+    kw.pop("mask")
+    parent = p.tree_parent.cuda()
+    mask = A.tree_mask(parent, p.tree_prefix, p.n_cells)
+    out.fill_(float("nan"))
+    args = A.make_args(q, k, v, out, mask=mask, **{**kw, "n_slices": n_slices, "grid_order": grid_order})
+    ws = poisoned_workspace(A.workspace_size(args, A.OP_DECODE))
+    A.attn_decode_args(args, ws=ws)
+    torch.cuda.synchronize()
+    A.check_device_status()
+    return out, mask
+
+
+@pytest.mark.parametrize("width", WIDTHS)
+@pytest.mark.parametrize("visible", [33, 34, 8193])
+def test_tree_mask_equals_host_mask(cuda_lib, width, visible):
+    p = W.tree_decode(width=width, visible=visible, Hq=4, Hkv=1, D=64)
+    mask = A.tree_mask(p.tree_parent.cuda(), p.tree_prefix, p.n_cells)
+    torch.cuda.synchronize()
+    assert torch.equal(mask.cpu(), p.mask)
+
+
+@pytest.mark.parametrize("visible", KEYS)
+@pytest.mark.parametrize("width", WIDTHS)
+def test_tree_decode_contract_shapes(cuda_lib, width, visible):
+    p = W.tree_decode(seed=2000 + width * 7 + visible % 97, width=width, visible=visible, Hq=8, Hkv=2, D=128)
+    ref = oracle.attn(p)
+    for S in (0, 7):
+        out, _ = decode_tree(p, n_slices=S)
+        check(p, out, f"width={width} keys={visible} S={S}", ref=ref)
+
+
+def test_tree_decode_full_heads_orders_bit_identical(cuda_lib):
+    """The GQA decode heads (32 q / 8 KV, D 128) at width 16 over 32770 keys;
+    every grid order and repeated run gives the same bits."""
+    p = W.tree_decode(width=16, visible=32770)
+    ref = oracle.attn(p)
+    base, _ = decode_tree(p, n_slices=16)
+    check(p, base, "tree full heads", ref=ref)
+    for order in (0, 1):
+        again, _ = decode_tree(p, n_slices=16, grid_order=order)
+        assert torch.equal(base.view(torch.int16), again.view(torch.int16))
+    auto, _ = decode_tree(p)
+    check(p, auto, "tree full heads, balanced", ref=ref)
+
+
+def test_tree_mask_rejects_a_parent_that_is_not_smaller(cuda_lib):
+    """A parent index >= its child is not heap order: the kernel's own check
+    stops the walk and the device status word reports it."""
+    p = W.tree_decode(width=8, visible=100, Hq=4, Hkv=1, D=64)
+    parent = p.tree_parent.clone()
+    parent[5] = 6
+    A.tree_mask(parent.cuda(), p.tree_prefix, p.n_cells)
+    with pytest.raises(A.AttnError) as e:
+        A.check_device_status()
+    assert e.value.status == -1
+    A.check_device_status()   # the status word was cleared
