@@ -18,8 +18,9 @@
 //    paths: strix-llama.cpp PR #115 "Performance" discussion.)
 //  * prefill_kernel: one CTA per (row tile, two q heads of one KV group).  Both
 //    heads share every K and V tile, so each tile crosses L2 once per pair.
-//      warp 0       TMA producer: Q of both heads once, then K_j, V_j through
-//                   a 3-stage ring (128-byte swizzled boxes of 64 x 128).
+//      warp 0       TMA producer: Q of both heads once, then K_j into a
+//                   one-tile K buffer and V_j into a two-tile V ring
+//                   (128-byte swizzled boxes of 64 x 128).
 //      warp 1       allocates 512 TMEM columns and issues the MMAs:
 //                     S_i  (TMEM cols i*128 .. +128)  = Q_i K_j^T
 //                     O_i  (TMEM cols 256 + i*D ..)  += P_i V_j
@@ -191,7 +192,7 @@ struct PfLayout {
   static constexpr int BOX = 128 * 128;                  // one TMA box: 128 rows x 128 B (64 values)
   static constexpr int TILE = kPfRows * D * 2;           // a Q, K or V tile: D/64 boxes
   static constexpr int PTILE = kPfRows * kPfCells * 2;   // a P tile: two boxes
-  static constexpr int NS = 3;                           // K/V ring stages (one tile each)
+  static constexpr int NS = 3;                           // K/V stages (one tile each): K, V, V
   static constexpr int OFF_Q = 0;                        // [2 slots][TILE]
   static constexpr int OFF_P = OFF_Q + 2 * TILE;         // [2 slots][PTILE]
   static constexpr int OFF_KV = OFF_P + 2 * PTILE;       // [NS][TILE]
@@ -220,6 +221,14 @@ __device__ __forceinline__ unsigned char* pf_align1024(unsigned char* p) {
   const uint32_t a = smem_u32(p);
   return p + (((a + 1023u) & ~1023u) - a);
 }
+
+// K/V ring: stage 0 holds the K tile of the current cell tile (one buffer,
+// refilled as soon as every head's S of that tile has completed, so the next K
+// streams in during the softmax); stages 1 and 2 hold V, tile j in stage
+// 1 + (j & 1), refilled once P V two tiles back has completed.  Neither load
+// waits on the tensor core's most recent work.
+__device__ __forceinline__ int pf_vstage(int64_t j) { return 1 + (int)(j & 1); }
+__device__ __forceinline__ uint32_t pf_vparity(int64_t j) { return (uint32_t)((j >> 1) & 1); }
 
 // Bounded wait that also gives up as soon as another thread of the CTA has
 // raised the abort flag.
@@ -746,9 +755,8 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
 
     if (code == kTileMixedBadV) {
       // P V on the CUDA cores over this row's visible cells only.
-      const int64_t LV = 2 * (int64_t)j + 1;
-      const int stV = (int)(LV % NS);
-      if (!pf_wait_warp(&kv_full[stV], (uint32_t)((LV / NS) & 1), p.status, abort_flag)) { ok = false; break; }
+      const int stV = pf_vstage(j);
+      if (!pf_wait_warp(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
       const unsigned char* Vs = sm + L::OFF_KV + stV * L::TILE;
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -896,8 +904,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
       int kt = tiles.first();
-      int64_t Lc = 0;   // loads issued into the ring
-      bool ok = true;
+      int64_t nK = 0, nV = 0;   // K and V tile loads issued
       const bool any = kt >= 0;
       if (any) {
         mbar_arrive_expect_tx(q_full, (uint32_t)(n_slots * L::TILE));
@@ -907,24 +914,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, q_full, bx * 64, h0 + s, rt * kPfRows,
                         pol);
       }
-      for (; ok && kt >= 0; kt = tiles.next(kt)) {
-        for (int kv = 0; kv < 2; ++kv) {
-          const int st = (int)(Lc % NS);
-          if (Lc >= NS && !pf_wait(&kv_empty[st], (uint32_t)(((Lc / NS) + 1) & 1), p.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&kv_full[st], (uint32_t)L::TILE);
+      for (; kt >= 0; kt = tiles.next(kt)) {
+        // K of this tile once every head's S of the previous tile is done
+        if (nK >= 1 && !pf_wait(&kv_empty[0], (uint32_t)((nK - 1) & 1), p.status, abort_flag)) break;
+        mbar_arrive_expect_tx(&kv_full[0], (uint32_t)L::TILE);
 #pragma unroll
-          for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_3d(sm + L::OFF_KV + st * L::TILE + bx * L::BOX, kv ? &tmV : &tmK, &kv_full[st], bx * 64, g,
-                        kt * kPfCells, pol);
-          ++Lc;
-        }
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(sm + L::OFF_KV + bx * L::BOX, &tmK, &kv_full[0], bx * 64, g, kt * kPfCells, pol);
+        ++nK;
+        // V of this tile once P V two tiles back is done
+        const int sv = pf_vstage(nV);
+        if (nV >= 2 && !pf_wait(&kv_empty[sv], (uint32_t)(((nV >> 1) - 1) & 1), p.status, abort_flag)) break;
+        mbar_arrive_expect_tx(&kv_full[sv], (uint32_t)L::TILE);
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(sm + L::OFF_KV + sv * L::TILE + bx * L::BOX, &tmV, &kv_full[sv], bx * 64, g, kt * kPfCells,
+                      pol);
+        ++nV;
       }
       // leave no copy in flight (bounded; completed loads return at once)
-      for (int64_t k = Lc > NS ? Lc - NS : 0; k < Lc; ++k)
-        mbar_wait_bounded(&kv_full[k % NS], (uint32_t)((k / NS) & 1), nullptr);
+      if (nK >= 1) mbar_wait_bounded(&kv_full[0], (uint32_t)((nK - 1) & 1), nullptr);
+      for (int64_t k = nV > 2 ? nV - 2 : 0; k < nV; ++k)
+        mbar_wait_bounded(&kv_full[pf_vstage(k)], pf_vparity(k), nullptr);
       if (any) mbar_wait_bounded(q_full, 0, nullptr);
     }
   } else if (warp == 1) {
@@ -952,22 +963,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int kn = tiles.next(kt);
         const bool has_next = kn >= 0;
         const bool pv_mma = tiles.code(kt) != kTileMixedBadV;
-        const int64_t LK = 2 * (j + 1), LV = 2 * j + 1;
-        const int stK = (int)(LK % NS), stV = (int)(LV % NS);
-        if (has_next && !pf_wait(&kv_full[stK], (uint32_t)((LK / NS) & 1), p.status, abort_flag)) break;
-        if (!pf_wait(&kv_full[stV], (uint32_t)((LV / NS) & 1), p.status, abort_flag)) break;
-        tc_fence_after();
+        const int stV = pf_vstage(j);
         // per head: the next tile's scores as soon as the softmax has read
         // this tile's S, then this tile's P V
         for (int s = 0; s < n_slots && ok; ++s) {
           if (has_next) {
+            if (s == 0 && !pf_wait(&kv_full[0], (uint32_t)((j + 1) & 1), p.status, abort_flag)) { ok = false; break; }
             if (!pf_wait(&s_free[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr + stK * L::TILE, idS);
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr, idS);
             umma_commit(&s_full[s]);
-            if (s == n_slots - 1) umma_commit(&kv_empty[stK]);
+            if (s == n_slots - 1) umma_commit(&kv_empty[0]);
           }
           if (!pf_wait(&p_full[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
+          if (s == 0 && !pf_wait(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if (pv_mma)
             pf_issue_pv<D>(tmem + 256u + (uint32_t)s * D, p_addr + s * L::PTILE, kv_addr + stV * L::TILE, idO,
