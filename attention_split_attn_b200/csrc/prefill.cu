@@ -24,14 +24,16 @@
 //      warp 1       allocates 512 TMEM columns and issues the MMAs:
 //                     S_i  (TMEM cols i*128 .. +128)  = Q_i K_j^T
 //                     O_i  (TMEM cols 256 + i*D ..)  += P_i V_j
-//                   S_i of tile j+1 is issued as soon as warpgroup i has
-//                   read S_i of tile j, so the tensor core computes the next
-//                   scores while the softmax of this tile runs.
+//                   P_i lives in the first 64 columns of S_i (16-bit, two
+//                   values per column) and is the MMA's A operand straight
+//                   from tensor memory.  Per head the tensor core runs
+//                   P V(j), then S(j+1) over the same columns; while one
+//                   head's softmax runs, the tensor core works for the other.
 //      warps 2-5    softmax of head slot 0; warps 6-9: slot 1.  Thread t owns
 //                   query row t of the tile (TMEM lane t): it reads its row of
 //                   S with tcgen05.ld, applies the transforms, keeps the
-//                   running max m and sum l, writes P (16-bit) to shared
-//                   memory in the UMMA K-major 128-byte-swizzled layout, and
+//                   running max m and sum l, writes P (16-bit) over its row
+//                   of S in tensor memory, and
 //                   rescales its O row in TMEM only when the max grew by more
 //                   than ln 256 (lazy rescaling: the weights stay <= 256, and
 //                   m is the common reference of l and O, so the result is
@@ -191,14 +193,14 @@ template <int D>
 struct PfLayout {
   static constexpr int BOX = 128 * 128;                  // one TMA box: 128 rows x 128 B (64 values)
   static constexpr int TILE = kPfRows * D * 2;           // a Q, K or V tile: D/64 boxes
-  static constexpr int PTILE = kPfRows * kPfCells * 2;   // a P tile: two boxes
+  static constexpr int PTILE = kPfRows * kPfCells * 2;   // a P tile (CUDA-core P V only): two boxes
   static constexpr int NS = 3;                           // K/V stages (one tile each): K, V, V
   static constexpr int OFF_Q = 0;                        // [2 slots][TILE]
   static constexpr int OFF_P = OFF_Q + 2 * TILE;         // [2 slots][PTILE]
   static constexpr int OFF_KV = OFF_P + 2 * PTILE;       // [NS][TILE]
   static constexpr int OFF_BAR = OFF_KV + NS * TILE;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_done[2], mma_done
-  static constexpr int N_BAR = 1 + 2 * NS + 8 + 1;
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], mma_done
+  static constexpr int N_BAR = 1 + 2 * NS + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;   // TMEM base address, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
@@ -281,6 +283,18 @@ __device__ __forceinline__ void pf_issue_pv(uint32_t d_tmem, uint32_t p_base, ui
             umma_desc_sw128(v_base + (uint32_t)kk * 2048u, PfLayout<D>::BOX, 1024), idesc,
             (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+// The same with P in tensor memory: P (16-bit, two values per 32-bit column,
+// row i in lane i) sits in the first 64 columns of the head's S region; each
+// MMA takes 16 cells = 8 columns of it.
+template <int D>
+__device__ __forceinline__ void pf_issue_pv_ts(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_base, uint32_t idesc,
+                                               bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kPfCells / 16; ++kk)
+    umma_ts(d_tmem, p_tmem + (uint32_t)kk * 8u, umma_desc_sw128(v_base + (uint32_t)kk * 2048u, PfLayout<D>::BOX, 1024),
+            idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Cell tiles of one row tile, skipping the empty ones, from the LAST to the
@@ -588,9 +602,8 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
   constexpr int NS = L::NS;
   uint64_t* kv_full = bars + 1;
   uint64_t* s_full = bars + 1 + 2 * NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* pv_done = s_full + 6;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = s_full + 4;
   const int row_t = quarter * 32 + lane;
   const int r = rt * kPfRows + row_t;
   const bool rvalid = r < p.R;
@@ -672,8 +685,6 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       if (cap && !bounded && __any_sync(0xffffffffu, !(smax <= p.s_lim))) {
         fast = false;
       } else {
-        tc_fence_before();
-        mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
         const float boff = al == 1 ? C : 0.f, bstep = al == 1 ? 8.f * slope : 0.f;
         if (bits_tile) {
           const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
@@ -712,18 +723,12 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
         else if (al_t == 1) pf_transform_exact<1>(raw, x, p, nslope, A, rpf, cpos, mt);
         else pf_transform_exact<2>(raw, x, p, nslope, A, rpf, cpos, mt);
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[slot]);          // the tensor core may overwrite S now
       if (code != kTileFull) pf_visibility(x, vis, p, rv, rvalid, c0, mrow, mask_vec, al == 2, nslope, mt);
       pf_weights<KT>(x, 0.f, 0.f, mt, m, l, mneg2, pk, need, factor);
     }
 
-    // P V of the previous tile must be complete before its P buffer is
-    // overwritten and before O is rescaled.
-    if (j > 0) {
-      if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p.status, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-    }
+    // P V of the previous tile is complete: the tensor core issued it before
+    // this tile's S, and S's completion covers every MMA issued before it.
     if (j > 0 && code != kTileMixedBadV && __any_sync(0xffffffffu, need)) {
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -742,18 +747,17 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       tmem_wait_st();
     }
 
-    // P row in the K-major 128-byte-swizzled layout the MMA reads: cells
-    // 0-63 in the first box, 64-127 in the second; 16-byte chunk k of row t
-    // at chunk k ^ (t & 7).
-#pragma unroll
-    for (int k8 = 0; k8 < kPfCells / 8; ++k8) {
-      const uint4 w = make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
-      const uint32_t off = (uint32_t)(k8 >> 3) * L::BOX + (uint32_t)row_t * 128u +
-                           ((uint32_t)((k8 & 7) ^ (row_t & 7)) << 4);
-      *reinterpret_cast<uint4*>(Ps + off) = w;
-    }
-
     if (code == kTileMixedBadV) {
+      // P row in shared memory (K-major 128-byte-swizzled: cells 0-63 in the
+      // first box, 64-127 in the second; 16-byte chunk k of row t at chunk
+      // k ^ (t & 7)) for the CUDA-core P V below.
+#pragma unroll
+      for (int k8 = 0; k8 < kPfCells / 8; ++k8) {
+        const uint4 w = make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
+        const uint32_t off = (uint32_t)(k8 >> 3) * L::BOX + (uint32_t)row_t * 128u +
+                             ((uint32_t)((k8 & 7) ^ (row_t & 7)) << 4);
+        *reinterpret_cast<uint4*>(Ps + off) = w;
+      }
       // P V on the CUDA cores over this row's visible cells only.
       const int stV = pf_vstage(j);
       if (!pf_wait_warp(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
@@ -795,7 +799,10 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       }
       tmem_wait_st();
     } else {
-      fence_async_smem();   // P visible to the tensor core
+      // P into the first 64 columns of this head's S region (S is read)
+      tmem_st32(tS, pk);
+      tmem_st32(tS + 32, pk + 32);
+      tmem_wait_st();
     }
     tc_fence_before();
     mbar_arrive(&p_full[slot]);
@@ -853,10 +860,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = bars + 1 + NS;
   uint64_t* s_full = bars + 1 + 2 * NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* pv_done = s_full + 6;
-  uint64_t* mma_done = s_full + 8;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = s_full + 4;
+  uint64_t* mma_done = s_full + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
 
@@ -874,7 +880,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < NS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], kPfRows);
       mbar_init(&p_full[s], kPfRows);
       mbar_init(&pv_done[s], 1);
     }
@@ -944,7 +949,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr int bf = Storage<KT>::kDtype == ATTN_BF16 ? 1 : 0;
       constexpr uint32_t idS = umma_idesc_f16(kPfRows, kPfCells, bf, 0, 0);
       constexpr uint32_t idO = umma_idesc_f16(kPfRows, D, bf, 0, 1);
-      const uint32_t q_addr = smem_u32(sm + L::OFF_Q), p_addr = smem_u32(sm + L::OFF_P);
+      const uint32_t q_addr = smem_u32(sm + L::OFF_Q);
       const uint32_t kv_addr = smem_u32(sm + L::OFF_KV);
       int kt = tiles.first();
       bool ok = kt >= 0;
@@ -964,24 +969,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool has_next = kn >= 0;
         const bool pv_mma = tiles.code(kt) != kTileMixedBadV;
         const int stV = pf_vstage(j);
-        // per head: the next tile's scores as soon as the softmax has read
-        // this tile's S, then this tile's P V
+        // per head: P V of this tile (P in the head's S columns), then the
+        // next tile's S over them
         for (int s = 0; s < n_slots && ok; ++s) {
+          if (!pf_wait(&p_full[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
+          if (s == 0 && !pf_wait(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          if (pv_mma)
+            pf_issue_pv_ts<D>(tmem + 256u + (uint32_t)s * D, tmem + (uint32_t)s * 128u, kv_addr + stV * L::TILE,
+                              idO, j > 0);
+          umma_commit(&pv_done[s]);
           if (has_next) {
             if (s == 0 && !pf_wait(&kv_full[0], (uint32_t)((j + 1) & 1), p.status, abort_flag)) { ok = false; break; }
-            if (!pf_wait(&s_free[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
             pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr, idS);
             umma_commit(&s_full[s]);
             if (s == n_slots - 1) umma_commit(&kv_empty[0]);
           }
-          if (!pf_wait(&p_full[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
-          if (s == 0 && !pf_wait(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          if (pv_mma)
-            pf_issue_pv<D>(tmem + 256u + (uint32_t)s * D, p_addr + s * L::PTILE, kv_addr + stV * L::TILE, idO,
-                           j > 0);
-          umma_commit(&pv_done[s]);
         }
         if (!ok) break;
         umma_commit(&kv_empty[stV]);
