@@ -282,7 +282,7 @@ def run_ours(args, rank, world, local):
         "frac_of_hbm_peak": value / world / hbm_peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
-                     "kernel": "decode_plan_kernel + decode_stream_kernel (balanced split-K)",
+                     "kernel": "decode_stream_kernel + combine_kernel (balanced split-K; the stream kernel computes the row tile prefix)",
                      "kernel_ms": kmean_ms, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
