@@ -22,12 +22,13 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
 
-ATTN_F32, ATTN_F16, ATTN_BF16 = 0, 1, 2
+ATTN_F32, ATTN_F16, ATTN_BF16, ATTN_FP8_E4M3, ATTN_I8 = 0, 1, 2, 3, 4
 OP_DECODE, OP_SELECTED, OP_PREFILL = 0, 1, 2
 STATUS = {0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED",
           -3: "ATTN_ERR_WORKSPACE", -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_DEVICE_TIMEOUT"}
 
-_DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN_BF16}
+_DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN_BF16,
+          torch.float8_e4m3fn: ATTN_FP8_E4M3, torch.int8: ATTN_I8}
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
@@ -57,6 +58,7 @@ class AttnArgs(ctypes.Structure):
         ("alibi_slopes", ctypes.c_void_p), ("sinks", ctypes.c_void_p),
         ("n_slices", ctypes.c_int32), ("max_row_len", ctypes.c_int32),
         ("grid_order", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5),
+        ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p), ("scale_stride_cell", ctypes.c_int64),
     ]
 
 
@@ -136,8 +138,9 @@ def _check_i32(name, t, n):
 
 def make_args(q, k, v, out, *, scale, softcap=0.0, row_begin=None, row_end=None, cell_seq=None,
               row_seq=None, cell_pos=None, row_pos=None, causal=False, mask=None, alibi_slopes=None,
-              sinks=None, n_slices=0, max_row_len=0, grid_order=0):
-    """Fill an AttnArgs from CUDA tensors (q/out [R, Hq, D], k/v [N, Hkv, D])."""
+              sinks=None, n_slices=0, max_row_len=0, grid_order=0, k_scale=None, v_scale=None):
+    """Fill an AttnArgs from CUDA tensors (q/out [R, Hq, D], k/v [N, Hkv, D]; for
+    an e4m3 or int8 cache, k_scale/v_scale are float32 [N, Hkv])."""
     if q.dim() != 3 or k.dim() != 3 or v.dim() != 3 or out.dim() != 3:
         raise ValueError("q, out must be [rows, heads, dim] and k, v [cells, heads, dim]")
     if k.shape != v.shape or k.stride() != v.stride() or k.dtype != v.dtype:
@@ -169,6 +172,15 @@ def make_args(q, k, v, out, *, scale, softcap=0.0, row_begin=None, row_end=None,
             raise ValueError(f"{name} must be a contiguous float32 tensor of n_head_q entries")
         setattr(a, name, _ptr(t))
     a.n_slices, a.max_row_len, a.grid_order = int(n_slices), int(max_row_len), int(grid_order)
+    if (k_scale is None) != (v_scale is None):
+        raise ValueError("k_scale and v_scale must both be given or both be None")
+    if k_scale is not None:
+        for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+            if t.dtype != torch.float32 or t.dim() != 2 or t.shape[0] != N or t.shape[1] != Hkv or t.stride(1) != 1:
+                raise ValueError(f"{name} must be float32 [n_cells, n_head_kv] with contiguous heads")
+        if k_scale.stride(0) != v_scale.stride(0):
+            raise ValueError("k_scale and v_scale must share their cell stride")
+        a.k_scale, a.v_scale, a.scale_stride_cell = k_scale.data_ptr(), v_scale.data_ptr(), k_scale.stride(0)
     return a
 
 
@@ -361,6 +373,8 @@ def problem_kwargs(p, device="cuda", out=None):
               row_pos=dev(p.row_pos), causal=p.causal, mask=dev(p.mask),
               alibi_slopes=dev(p.alibi_slopes), sinks=dev(p.sinks), n_slices=p.n_slices,
               max_row_len=p.max_row_len)
+    if p.k_scale is not None:
+        kw["k_scale"], kw["v_scale"] = dev(p.k_scale), dev(p.v_scale)
     if p.sel is not None:
         for key in ("row_begin", "row_end", "cell_seq", "row_seq", "mask", "causal", "max_row_len"):
             kw.pop(key)

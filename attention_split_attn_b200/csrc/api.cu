@@ -41,6 +41,8 @@ int dtype_size(int32_t t) {
     case ATTN_F32: return 4;
     case ATTN_F16: return 2;
     case ATTN_BF16: return 2;
+    case ATTN_FP8_E4M3: return 1;
+    case ATTN_I8: return 1;
     default: return 0;
   }
 }
@@ -113,6 +115,8 @@ CUtensorMapDataType tma_dtype(int32_t t) {
   switch (t) {
     case ATTN_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     case ATTN_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    case ATTN_FP8_E4M3:
+    case ATTN_I8: return CU_TENSOR_MAP_DATA_TYPE_UINT8;   // raw codes; the kernel decodes them
     default: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   }
 }
@@ -143,6 +147,8 @@ int32_t make_kv_map(CUtensorMap* map, const void* base, int32_t type, int D, int
 // ---- validation ----------------------------------------------------------------
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool is_quantized(int32_t t) { return t == ATTN_FP8_E4M3 || t == ATTN_I8; }
+
 int32_t validate_common(const attn_args* a, int32_t op) {
   if (!a) return fail(ATTN_ERR_INVALID_ARG, "args is NULL");
   for (int i = 0; i < 5; ++i)
@@ -155,6 +161,18 @@ int32_t validate_common(const attn_args* a, int32_t op) {
                 a->n_head_kv);
   if (!dtype_size(a->q_type) || !dtype_size(a->kv_type) || !dtype_size(a->out_type))
     return fail(ATTN_ERR_INVALID_ARG, "unknown dtype");
+  if (is_quantized(a->q_type) || is_quantized(a->out_type))
+    return fail(ATTN_ERR_UNSUPPORTED, "Q and out cannot be e4m3 or int8 (only the K/V cache can)");
+  if (is_quantized(a->kv_type)) {
+    if (op != ATTN_OP_DECODE)
+      return fail(ATTN_ERR_UNSUPPORTED, "e4m3/int8 K/V caches are supported by attn_decode only");
+    if (a->n_cells > 0 && (!a->k_scale || !a->v_scale))
+      return fail(ATTN_ERR_INVALID_ARG, "an e4m3/int8 cache needs k_scale and v_scale");
+    if (a->n_cells > 1 && a->scale_stride_cell < a->n_head_kv)
+      return fail(ATTN_ERR_INVALID_ARG, "scale_stride_cell is smaller than n_head_kv");
+  } else if (a->k_scale || a->v_scale) {
+    return fail(ATTN_ERR_INVALID_ARG, "k_scale/v_scale are only for e4m3/int8 caches");
+  }
   if (a->head_dim != 64 && a->head_dim != 128 && a->head_dim != 256)
     return fail(ATTN_ERR_UNSUPPORTED, "head_dim %d not in {64, 128, 256}", a->head_dim);
   const int G = a->n_head_q / a->n_head_kv;
@@ -184,7 +202,6 @@ int32_t validate_common(const attn_args* a, int32_t op) {
     if ((a->n_cells > 1 && a->kv_stride_cell == 0) || (a->n_head_kv > 1 && a->kv_stride_head == 0))
       return fail(ATTN_ERR_UNSUPPORTED, "zero kv stride (broadcast caches are not supported)");
   }
-  (void)op;
   return ATTN_OK;
 }
 
@@ -554,6 +571,7 @@ int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* s
   p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
   p.S = sh.S; p.C = sh.C; p.grid_order = a->grid_order;
   p.hpw = sh.hpw; p.hg = sh.hg; p.kv_type = a->kv_type; p.mma = mma ? 1 : 0;
+  p.k_scale = a->k_scale; p.v_scale = a->v_scale; p.scale_sc = a->scale_stride_cell;
   p.status = di->status;
   const DecodeWs wl = decode_ws_layout(a, sh);
   char* wsb = static_cast<char*>(ws);

@@ -1,5 +1,6 @@
 // decode_slice.cu -- split-K decode attention on a (rows, heads, slices) grid
-// (attn_decode with a forced slice count, and every FP32 or mixed-dtype cache).
+// (attn_decode with a forced slice count, every FP32 or mixed-dtype cache, and
+// the e4m3 / int8 caches with per (cell, KV head) scales).
 //
 // Work decomposition (TensorFold PR #2595, "What this changes": the
 // attn_decode grid is (rows, heads, slices) so that rows sharing a key slice
@@ -82,6 +83,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   using Geo = DecodeGeom<KT, D>;
   using Sm = DecodeSmem<KT, D, HPW, HG>;
   constexpr int NCW = kKeyWarps * HG;
+  constexpr bool kQuant = Storage<KT>::kDtype == ATTN_FP8_E4M3 || Storage<KT>::kDtype == ATTN_I8;
   constexpr int NS = Geo::NSTAGE;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::kBarOffset);
@@ -251,9 +253,11 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll
         for (int h = 0; h < HPW; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], off);
       const float negdist = -(float)(rc.row_pos >= cpos ? rc.row_pos - cpos : cpos - rc.row_pos);
+      // quantized cache: q.(s_k code) = s_k (q.code), the dequantized dot product
+      const float ks = kQuant ? (vk ? __ldg(p.k_scale + (int64_t)c * p.scale_sc + g) : 0.f) : 1.f;
 #pragma unroll
       for (int h = 0; h < HPW; ++h) {
-        float xv = acc[h];
+        float xv = kQuant ? acc[h] * ks : acc[h];
         if (softcap > 0.f) xv = softcap * tanhf(xv / softcap);
         if (alibi) xv = fmaf(slope[h], negdist, xv);
         xv += mval;
@@ -285,12 +289,15 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (!vis[i]) w = make_uint4(0u, 0u, 0u, 0u);
         unpack_vec<KT>(w, vf + v * Geo::EPV);
       }
+      // quantized cache: p (s_v code) = (p s_v) code
+      const float vs = kQuant ? (vis[i] ? __ldg(p.v_scale + (int64_t)(tile0 + j) * p.scale_sc + g) : 0.f) : 1.f;
 #pragma unroll
       for (int h = 0; h < HPW; ++h) {
         const float pr = ex2((x[i][h] - mu[h]) * kLog2e);
         l[h] += pr;
+        const float pv = kQuant ? pr * vs : pr;
 #pragma unroll
-        for (int e = 0; e < Geo::EPL; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
+        for (int e = 0; e < Geo::EPL; ++e) o[h][e] = fmaf(pv, vf[e], o[h][e]);
       }
     }
     __syncwarp();
@@ -527,7 +534,8 @@ bool decode_uses_mma(int kv_type, int q_type, const void* q, int64_t q_sr, int64
 }
 
 bool decode_shape_supported(int kv_type, int D, int G) {
-  return (kv_type == ATTN_F32 || kv_type == ATTN_F16 || kv_type == ATTN_BF16) &&
+  return (kv_type == ATTN_F32 || kv_type == ATTN_F16 || kv_type == ATTN_BF16 || kv_type == ATTN_FP8_E4M3 ||
+          kv_type == ATTN_I8) &&
          (D == 64 || D == 128 || D == 256) && G >= 1 && G <= 16;
 }
 
@@ -540,6 +548,8 @@ cudaError_t launch_decode_slices(const DecodePlan& p, const CUtensorMap& tmK, co
   switch (p.kv_type) {
     case ATTN_F32: return launch_decode_k<float>(p, tmK, tmV, stream);
     case ATTN_F16: return launch_decode_k<__half>(p, tmK, tmV, stream);
+    case ATTN_FP8_E4M3: return launch_decode_k<e4m3_code>(p, tmK, tmV, stream);
+    case ATTN_I8: return launch_decode_k<i8_code>(p, tmK, tmV, stream);
     default: return launch_decode_k<__nv_bfloat16>(p, tmK, tmV, stream);
   }
 }

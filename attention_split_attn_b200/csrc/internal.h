@@ -65,6 +65,9 @@ struct DecodePlan {
   int32_t W;          // warps of the persistent grid
   int64_t* row_tiles; // [R+1] exclusive prefix of 16-cell tiles per row (planner output)
   int32_t plan_inline; // 1: few rows; the stream kernel computes the prefix (no planner)
+  // e4m3 / int8 caches: per (cell, KV head) scales at c * scale_sc + g
+  const float *k_scale, *v_scale;
+  int64_t scale_sc;
 };
 
 bool decode_uses_mma(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh);

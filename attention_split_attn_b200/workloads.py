@@ -57,6 +57,8 @@ class Problem:
     sel: Optional[torch.Tensor] = None         # int32 [R, n_sel]
     n_slices: int = 0                          # 0: chosen by the planner
     max_row_len: int = 0                       # 0: unknown (bounded by N)
+    k_scale: Optional[torch.Tensor] = None     # float32 [N, Hkv] (e4m3 / int8 caches)
+    v_scale: Optional[torch.Tensor] = None     # float32 [N, Hkv]
 
     @property
     def n_rows(self) -> int: return self.q.shape[0]
@@ -126,6 +128,35 @@ def gqa_decode(seed: int = 1002, n_seq: int = 16, cap: int = 8192, Hq: int = 32,
     begin = np.arange(n_seq, dtype=np.int64) * cap
     return Problem("gqa_decode", q, k, v, out_dtype=BF16, scale=1.0 / math.sqrt(D),
                    row_begin=_i32(begin), row_end=_i32(begin + lens), max_row_len=cap)
+
+
+def quantize_kv(x: torch.Tensor, fmt: str):
+    """Codes and float32 [N, Hkv] scales of a float [N, Hkv, D] cache: one scale
+    per (cell, KV head) = amax / 448 for e4m3 (TensorFold PR #911), amax / 127
+    for int8; an all-zero row gets scale 1."""
+    amax = x.abs().amax(dim=2).to(torch.float32)
+    top = 448.0 if fmt == "e4m3" else 127.0
+    scale = torch.where(amax > 0, amax / top, torch.ones_like(amax))
+    y = x.to(torch.float32) / scale[:, :, None]
+    if fmt == "e4m3":
+        return y.to(torch.float8_e4m3fn), scale
+    return torch.round(y).clamp(-127, 127).to(torch.int8), scale
+
+
+def quantized_decode(seed: int = 1007, fmt: str = "e4m3", n_seq: int = 16, cap: int = 8192, Hq: int = 32,
+                     Hkv: int = 8, D: int = 128) -> Problem:
+    """The GQA decode batch (16 sequences x 1 row, 32/8 heads, D 128, len_s ~
+    U{1024..8192} in a [16*8192, 8, 128] cache) over an e4m3 or int8 cache
+    quantized from N(0,1) rows with per (cell, KV head) scales; bf16 Q and out."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(min(1024, cap), cap + 1, size=n_seq)
+    N = n_seq * cap
+    q = _normal(rng, (n_seq, Hq, D), BF16)
+    k, ks = quantize_kv(_normal(rng, (N, Hkv, D), F32), fmt)
+    v, vs = quantize_kv(_normal(rng, (N, Hkv, D), F32), fmt)
+    begin = np.arange(n_seq, dtype=np.int64) * cap
+    return Problem(f"quantized_decode_{fmt}", q, k, v, out_dtype=BF16, scale=1.0 / math.sqrt(D),
+                   row_begin=_i32(begin), row_end=_i32(begin + lens), max_row_len=cap, k_scale=ks, v_scale=vs)
 
 
 def selected_prefill(seed: int = 1003, R: int = 2048, N: int = 32768, Hq: int = 48,

@@ -461,6 +461,34 @@ def run_parts(args, rank, dev, stream):
     }
     del q, k, v, out, ta, ws, kw, tmask
 
+    # quantized GQA decode: the decode batch's shape (16 rows, lengths U[1024,
+    # 8192], Hq 32 / Hkv 8, D 128) over an e4m3 cache with one F32 scale per
+    # (cell, KV head) for K and for V (TensorFold PR #911).  Bytes: the K and V
+    # codes and scales of every visible (cell, KV head), Q and out.
+    p = W.quantized_decode(fmt="e4m3")
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    qa = A.make_args(q, k, v, out, **kw)
+    qws_n = A.workspace_size(qa, A.OP_DECODE)
+    ws = torch.empty(max(qws_n, 256), dtype=torch.uint8, device=dev)
+    lens = int((p.row_end - p.row_begin).to(torch.int64).sum())
+    qbytes = (lens * p.n_head_kv * (2 * p.head_dim + 2 * 4) + p.q.numel() * p.q.element_size()
+              + p.n_rows * p.n_head_q * p.head_dim * 2)
+    for _ in range(max(args.warmup, 3)):
+        A.attn_decode_args(qa, ws=ws, stream=stream)
+    whole, main = _time_calls(lambda e: A.attn_decode_timed_args(qa, ws, e, stream=stream), n, flush, stream)
+    parts["fp8_decode"] = {
+        "workload": "quantized_decode: 16 seq x 1 row, Hq 32 / Hkv 8, D 128, e4m3 KV with per (cell, KV head) "
+                    "F32 scales, len U[1024,8192], bf16 out",
+        "value": qbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (visible K/V codes + scales, Q, out)",
+        "ms_per_call": whole, "calls": n,
+        "gpu_launches": (2 if qws_n > 0 else 1) * n,   # slice kernel (+ split_k_reduce)
+        "roofline": {"bound": "hbm", "achieved": qbytes / (main * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": qbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None, "kernel_ms": main,
+                     "algorithmic_bytes": qbytes, "kernel": "decode_slice_kernel<e4m3> (+ combine_kernel)",
+                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
+    }
+    del q, k, v, out, qa, ws, kw
+
     # semantics sweep: unified fp16 cache of 8 interleaved sequences, 256 rows,
     # per-cell sequence ids and positions, F32 mask, NaN cells, sinks; through
     # attn_decode (planner slices) and attn_prefill.  Bytes: the K and V rows of

@@ -83,6 +83,19 @@
  *   mask [n_rows][n_cells] F32            mask_stride_row
  * K and V base addresses and their cell/head strides must be 16-byte
  * aligned (tile loads by the Tensor Memory Accelerator).
+ *
+ * Quantized caches (attn_decode only; TensorFold PR #911: e4m3 rows with one
+ * fp32 scale per (position, key head) = amax / 448, half the bytes of bf16;
+ * TensorFold PR #2595: an int8 cache with a K scale and a V scale per key).
+ * With kv_type ATTN_FP8_E4M3 or ATTN_I8 the stored codes are one byte each and
+ *   k_c[d] = k_scale[c * scale_stride_cell + g] * code(K[c][g][d]),
+ *   v_c[d] = v_scale[c * scale_stride_cell + g] * code(V[c][g][d]),
+ * with code() the OCP FP8 E4M3 value (bias 7, no infinities, S.1111.111 is
+ * NaN) or the two's-complement int8 value; everything else is as above on the
+ * dequantized K/V.  Strides stay in elements (= bytes).  k_scale, v_scale:
+ * F32 device arrays, non-NULL for a quantized cache with n_cells > 0 and NULL
+ * otherwise; scale_stride_cell >= n_head_kv.  Q and out are never quantized.
+ * attn_selected and attn_prefill refuse quantized caches (ATTN_ERR_UNSUPPORTED).
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -94,9 +107,9 @@
 extern "C" {
 #endif
 
-#define ATTN_ABI_VERSION 1
+#define ATTN_ABI_VERSION 2
 
-typedef enum { ATTN_F32 = 0, ATTN_F16 = 1, ATTN_BF16 = 2 } attn_dtype;
+typedef enum { ATTN_F32 = 0, ATTN_F16 = 1, ATTN_BF16 = 2, ATTN_FP8_E4M3 = 3, ATTN_I8 = 4 } attn_dtype;
 
 typedef enum {
     ATTN_OK = 0,
@@ -138,6 +151,9 @@ typedef struct {
                              grid; 1: slices fastest.  Results are bit-identical;
                              exposed for tests and tuning.                           */
     int32_t reserved[5];  /* must be zero                                            */
+
+    const float *k_scale, *v_scale;   /* quantized caches: per (cell, KV head) scales, else NULL */
+    int64_t scale_stride_cell;        /* elements between cells' scale rows (>= n_head_kv)   */
 } attn_args;
 
 /* Selected-key arguments.  base.row_begin/row_end/cell_seq/row_seq/mask must be

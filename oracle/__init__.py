@@ -94,6 +94,33 @@ def _i32(t):
     return None if t is None else np.ascontiguousarray(t.numpy().astype(np.int32))
 
 
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    """float64 value of OCP FP8 E4M3 codes (uint8), from the format's definition:
+    1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 is
+    subnormal (m/8 * 2^-6); there are no infinities, and exponent 15 with
+    mantissa 7 is NaN.  (The e4m3 KV cache of TensorFold PR #911.)"""
+    c = codes.astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    val = np.where((e == 15) & (c & 0x7 == 7), np.nan, val)
+    return sign * val
+
+
+def _kv64(t, scale):
+    """A K or V cache widened to float64; an e4m3 or int8 cache is dequantized
+    as code times its (cell, KV head) scale (TensorFold PR #911: one fp32 scale
+    per position and key head; TensorFold PR #2595: K and V scales per key)."""
+    if t.dtype == torch.float8_e4m3fn:
+        code = e4m3_value(t.view(torch.uint8).numpy())
+    elif t.dtype == torch.int8:
+        code = t.numpy().astype(np.float64)
+    else:
+        return _f64(t)
+    return np.ascontiguousarray(code * scale.numpy().astype(np.float64)[:, :, None])
+
+
 def _f32(t):
     return None if t is None else np.ascontiguousarray(t.numpy().astype(np.float32))
 
@@ -104,7 +131,7 @@ def _ptr(a):
 
 def _marshal(p):
     keep = {
-        "q": _f64(p.q), "k": _f64(p.k), "v": _f64(p.v),
+        "q": _f64(p.q), "k": _kv64(p.k, p.k_scale), "v": _kv64(p.v, p.v_scale),
         "row_begin": _i32(p.row_begin), "row_end": _i32(p.row_end),
         "cell_seq": _i32(p.cell_seq), "row_seq": _i32(p.row_seq),
         "cell_pos": _i32(p.cell_pos), "row_pos": _i32(p.row_pos),

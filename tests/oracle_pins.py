@@ -12,7 +12,8 @@ what the pages or the mathematics fix.  The pins use:
     inputs;
   * invariants (selection duplicates and order, unified-cache isolation, the
     split form, full selection == dense causal);
-  * numpy.unique for the selection compaction.
+  * numpy.unique for the selection compaction;
+  * torch's float8_e4m3fn conversion for the e4m3 codes of a quantized cache.
 test_oracle_pins.py runs each one; test_oracle_mutations.py plants each known
 kind of mistake in the oracle and checks that some pin catches it.
 """
@@ -442,6 +443,47 @@ def pin_split_form_equals_plain():
             _close(got, ref, rtol=1e-14, atol=1e-15)
             z = (ref == 0)
             assert np.array_equal(got[z], ref[z]) and not np.signbit(got[z]).any()
+
+
+# ----------------------------------------------------------------------------
+# Quantized caches (e4m3 / int8 codes with per (cell, KV head) scales)
+# ----------------------------------------------------------------------------
+
+def pin_e4m3_codes_match_torch():
+    """The oracle's E4M3 decoding, written from the format's definition, against
+    torch's float8_e4m3fn conversion for all 256 codes (NaN codes included)."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_value(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    assert np.signbit(mine[0x80]) and mine[0x80] == 0 and mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9
+
+
+def pin_quantized_cache_equals_dequantized_sdpa():
+    """An e4m3 or int8 cache with scales that differ across cells and KV heads
+    (a scale applied to the wrong cell, head or tensor changes the result) is
+    SDPA over the cache dequantized by torch (code * scale) in float64."""
+    for fmt in ("e4m3", "i8"):
+        for seed in range(3):
+            rng = np.random.default_rng(700 + seed)
+            R, Hq, Hkv, D, N = 3, 4, 2, 16, 40
+            q = torch.from_numpy(rng.standard_normal((R, Hq, D)).astype(np.float32))
+            raw_k = torch.from_numpy((rng.standard_normal((N, Hkv, D)) *
+                                      rng.uniform(0.1, 8.0, (N, Hkv, 1))).astype(np.float32))
+            raw_v = torch.from_numpy((rng.standard_normal((N, Hkv, D)) *
+                                      rng.uniform(0.1, 8.0, (N, Hkv, 1))).astype(np.float32))
+            k, ks = W.quantize_kv(raw_k, fmt)
+            v, vs = W.quantize_kv(raw_v, fmt)
+            pq = W.Problem("quant_pin", q, k, v, scale=0.3, k_scale=ks, v_scale=vs,
+                           row_begin=torch.tensor([0, 5, 11], dtype=torch.int32),
+                           row_end=torch.tensor([40, 33, 12], dtype=torch.int32),
+                           sinks=torch.tensor([0.5, -1.0, -INF, 2.0], dtype=torch.float32))
+            deq = lambda c, sc: c.to(torch.float64) * sc.to(torch.float64)[:, :, None]
+            pd = dataclasses.replace(pq, k=deq(k, ks), v=deq(v, vs), k_scale=None, v_scale=None)
+            ref, _ = sdpa_reference(pd)
+            _close(oracle.attn(pq), ref, rtol=1e-12, atol=1e-14)
 
 
 PINS = {name: fn for name, fn in globals().items() if name.startswith("pin_") and callable(fn)}

@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version(lib):
-    assert lib.attn_abi_version() == 1
+    assert lib.attn_abi_version() == 2
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -113,6 +113,23 @@ def test_validation_pairs_and_reserved(lib):
     a = _args()
     a.reserved[2] = 1
     assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1
+
+
+def test_quantized_cache_validation(lib):
+    """e4m3/int8 caches: decode only, scales required, and only for such caches."""
+    for kv in (A.ATTN_FP8_E4M3, A.ATTN_I8):
+        a = _args(kv_type=kv, kv_stride_cell=2 * 128, kv_stride_head=128)
+        assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1      # scales missing
+        a.k_scale, a.v_scale, a.scale_stride_cell = 0x60000, 0x70000, a.n_head_kv
+        assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == 0
+        assert lib.attn_supports(ctypes.byref(a), A.OP_PREFILL) == -2
+        a.scale_stride_cell = a.n_head_kv - 1
+        assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1
+    a = _args()
+    a.k_scale, a.v_scale, a.scale_stride_cell = 0x60000, 0x70000, 8
+    assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1          # 16/32-bit cache with scales
+    a = _args(q_type=A.ATTN_FP8_E4M3)
+    assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -2          # Q is never quantized
 
 
 def test_empty_problem_is_ok(lib):
