@@ -5,8 +5,8 @@
 Workload: GQA split-K decode -- 16 sequences x 1 query row, 32 query heads over
 8 KV heads, head_dim 128, bf16 KV cache [16 x 8192 cells, 8, 128] with
 per-sequence lengths uniform in [1024, 8192] (seed 1002), bf16 output, slice
-count from the planner.  One step = one attn_decode call (slice kernel +
-split_k_reduce) over one batch.  The metric is attention GB/s: the algorithmic
+count from the planner.  One step = one attn_decode call (the balanced
+stream kernel + split_k_reduce) over one batch.  The metric is attention GB/s: the algorithmic
 bytes of a step (K and V rows of every visible cell, Q and the output) over
 the step time, with the HBM roofline of the dominant kernel beside it.
 
@@ -20,8 +20,9 @@ workloads, per call with the L2 flushed before each call: maskless
 selected-key attention (2048 rows, GQA 12, D 256, fp16 cache of 32768 cells;
 effective GB/s of the gathered K/V rows) and causal prefill (2048 rows over
 14048 cells, Hq 64 / Hkv 8, D 128, bf16; TFLOP/s over the visible pairs on
-the tensor cores), draft-tree decode rows (tree mask + attn_decode), and the
-unified-cache semantics sweep through attn_decode and attn_prefill (GB/s of the
+the tensor cores), draft-tree decode rows (tree mask + attn_decode), the
+decode batch over an e4m3 cache with per (cell, KV head) scales (GB/s of the
+visible codes and scales, Q and out), and the unified-cache semantics sweep through attn_decode and attn_prefill (GB/s of the
 visible K/V rows, mask rows and cell metadata), each with the roofline of its
 main kernel.
 --profile-op {decode,selected,prefill,semantics} only runs W + K calls of one operation
