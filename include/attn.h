@@ -10,7 +10,10 @@
  *                  slice partials.  Defined by TensorFold PR #2595 ("attn_decode
  *                  grid becomes (rows, heads, slices)"; attn_decode + attn_merge
  *                  registered as one operator: Q rows, K/V cache -> attention
- *                  rows; 32-key slices).
+ *                  rows; 32-key slices).  Supported: K/V in F32, F16, BF16,
+ *                  or e4m3 / int8 codes with scales (see "Quantized caches"
+ *                  below); Q in F32, F16 or BF16; head_dim 64, 128 or 256;
+ *                  1 to 16 query heads per KV head; any out dtype.
  *   attn_selected  maskless selected-key attention: a query row sees exactly
  *                  the cells named in its selection list; the list is sorted,
  *                  invalid and duplicate entries are skipped, and K/V are

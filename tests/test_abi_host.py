@@ -137,6 +137,21 @@ def test_empty_problem_is_ok(lib):
     assert lib.attn_decode(ctypes.byref(a), None, 0, None) == 0
 
 
+def test_quantized_decode_slice_plan(lib):
+    """e4m3/int8 caches take 2048-cell slices: 8192-cell rows -> 4 slices,
+    R * Hq * 4 partial records of D + 2 floats."""
+    a = _args(n_rows=16, n_head_q=32, n_head_kv=8, n_cells=131072, max_row_len=8192,
+              kv_type=A.ATTN_FP8_E4M3, kv_stride_cell=8 * 128, kv_stride_head=128)
+    a.k_scale, a.v_scale, a.scale_stride_cell = 0x60000, 0x70000, 8
+    ws = lib.attn_workspace_size(ctypes.byref(a), A.OP_DECODE, 0)
+    slots = 16 * 32 * 4
+    assert ws == (slots * 128 * 4 + 255) // 256 * 256 + (slots * 2 * 4 + 255) // 256 * 256
+    a.n_slices = 3                 # a forced count still wins
+    ws = lib.attn_workspace_size(ctypes.byref(a), A.OP_DECODE, 0)
+    slots = 16 * 32 * 3
+    assert ws == (slots * 128 * 4 + 255) // 256 * 256 + (slots * 2 * 4 + 255) // 256 * 256
+
+
 def test_strerror(lib):
     for code, name in A.STATUS.items():
         assert lib.attn_strerror(code).decode() == name
