@@ -34,7 +34,11 @@ MUTATIONS = {
     "empty_row_nan": 5, "gqa_modulo": 6, "no_dedup": 7, "mask_narrowed": 8,
     "invalid_clamped": 9, "scale_after_cap": 10, "neg_inf_mask_added": 11,
     "causal_strict": 12, "seq_ignored": 13, "k_d_reversed": 14,
+    # planted in the dequantization of e4m3 / int8 caches below (Python side)
+    "e4m3_bias_8": 101, "e4m3_nan_as_number": 102, "scale_cells_reversed": 103,
+    "scale_heads_reversed": 104, "k_scale_for_v": 105, "int8_as_unsigned": 106,
 }
+_py_mutation = 0   # the planted dequantization mistake in force (0: none)
 
 
 def build(force: bool = False) -> str:
@@ -103,8 +107,10 @@ def e4m3_value(codes: np.ndarray) -> np.ndarray:
     sign = np.where(c & 0x80, -1.0, 1.0)
     e = (c >> 3) & 0xF
     m = (c & 0x7).astype(np.float64)
-    val = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
-    val = np.where((e == 15) & (c & 0x7 == 7), np.nan, val)
+    bias = 8 if _py_mutation == MUTATIONS["e4m3_bias_8"] else 7
+    val = np.where(e == 0, np.ldexp(m / 8.0, 1 - bias), np.ldexp(1.0 + m / 8.0, e - bias))
+    if _py_mutation != MUTATIONS["e4m3_nan_as_number"]:
+        val = np.where((e == 15) & (c & 0x7 == 7), np.nan, val)
     return sign * val
 
 
@@ -116,9 +122,16 @@ def _kv64(t, scale):
         code = e4m3_value(t.view(torch.uint8).numpy())
     elif t.dtype == torch.int8:
         code = t.numpy().astype(np.float64)
+        if _py_mutation == MUTATIONS["int8_as_unsigned"]:
+            code = t.view(torch.uint8).numpy().astype(np.float64)
     else:
         return _f64(t)
-    return np.ascontiguousarray(code * scale.numpy().astype(np.float64)[:, :, None])
+    sc = scale.numpy().astype(np.float64)
+    if _py_mutation == MUTATIONS["scale_cells_reversed"]:
+        sc = sc[::-1]
+    if _py_mutation == MUTATIONS["scale_heads_reversed"]:
+        sc = sc[:, ::-1]
+    return np.ascontiguousarray(code * sc[:, :, None])
 
 
 def _f32(t):
@@ -131,7 +144,8 @@ def _ptr(a):
 
 def _marshal(p):
     keep = {
-        "q": _f64(p.q), "k": _kv64(p.k, p.k_scale), "v": _kv64(p.v, p.v_scale),
+        "q": _f64(p.q), "k": _kv64(p.k, p.k_scale),
+        "v": _kv64(p.v, p.k_scale if _py_mutation == MUTATIONS["k_scale_for_v"] else p.v_scale),
         "row_begin": _i32(p.row_begin), "row_end": _i32(p.row_end),
         "cell_seq": _i32(p.cell_seq), "row_seq": _i32(p.row_seq),
         "cell_pos": _i32(p.cell_pos), "row_pos": _i32(p.row_pos),
@@ -208,9 +222,15 @@ class mutation:
         self.code = MUTATIONS[name]
 
     def __enter__(self):
-        _load().oracle_set_mutation(self.code)
+        global _py_mutation
+        if self.code >= 100:
+            _py_mutation = self.code
+        else:
+            _load().oracle_set_mutation(self.code)
         return self
 
     def __exit__(self, *exc):
+        global _py_mutation
+        _py_mutation = 0
         _load().oracle_set_mutation(0)
         return False

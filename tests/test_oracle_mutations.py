@@ -4,8 +4,11 @@ Each mutation is a plausible slip named in the pages' own bug reports (ALiBi
 before softcap, NaN turned into 0, an unguarded exp(-inf - -inf) on an empty
 row, a narrowed F16 mask -- HartsyInference PR #910; duplicate or invalid
 selection entries not skipped -- strix-llama.cpp PR #115/#119) or a generic one
-(wrong sign, wrong GQA index, reversed operand, off-by-one causality).  The
-mistake is planted in the oracle, on the CPU, and the pin suite must go red.
+(wrong sign, wrong GQA index, reversed operand, off-by-one causality), or a
+slip in the dequantization of an e4m3 / int8 cache (wrong exponent bias, the
+NaN code read as a number, a scale taken from the wrong cell, head or tensor,
+int8 read unsigned).  The mistake is planted in the oracle, on the CPU, and the
+pin suite must go red.
 """
 import pytest
 
