@@ -8,8 +8,10 @@ with it: the only thing both sides use is the seeded input generator module
 
 The C library (``oracle.c``) is compiled with gcc, without fast-math, the
 first time it is needed (or by ``build()``).  Inputs are widened exactly to
-float64 here (every f16/bf16/f32 value is exactly representable in f64) and
-the result is returned in float64, before any rounding to an output dtype.
+float64 here (every f16/bf16/f32 value is exactly representable in f64); the
+codes of an e4m3 or int8 cache are dequantized here as code times the cell's
+and KV head's scale, in float64, before the C definition sees them.  The
+result is returned in float64, before any rounding to an output dtype.
 """
 from __future__ import annotations
 
