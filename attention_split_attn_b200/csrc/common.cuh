@@ -89,21 +89,6 @@ template <typename T> struct Storage;
 template <> struct Storage<float> { static constexpr int kDtype = ATTN_F32; };
 template <> struct Storage<__half> { static constexpr int kDtype = ATTN_F16; };
 template <> struct Storage<__nv_bfloat16> { static constexpr int kDtype = ATTN_BF16; };
-// One-byte codes of a quantized cache (the value is the code times a scale).
-struct e4m3_code { uint8_t bits; };
-struct i8_code { int8_t bits; };
-template <> struct Storage<e4m3_code> { static constexpr int kDtype = ATTN_FP8_E4M3; };
-template <> struct Storage<i8_code> { static constexpr int kDtype = ATTN_I8; };
-
-// Two e4m3 codes (low byte first) to floats, by the hardware conversion to
-// f16x2 (exact: every e4m3 value is an f16 value; S.1111.111 gives NaN).
-__device__ __forceinline__ void unpack_e4m3x2(uint32_t two, float& lo, float& hi) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(two & 0xffffu)));
-  const float2 f = __half22float2(*reinterpret_cast<__half2*>(&h2));
-  lo = f.x;
-  hi = f.y;
-}
 
 __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
   lo = __uint_as_float(w << 16);
@@ -117,20 +102,7 @@ __device__ __forceinline__ void unpack_f16x2(uint32_t w, float& lo, float& hi) {
 
 template <typename T>
 __device__ __forceinline__ void unpack_vec(const uint4& w, float* f) {
-  if constexpr (Storage<T>::kDtype == ATTN_FP8_E4M3) {
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      unpack_e4m3x2(ws[k], f[4 * k], f[4 * k + 1]);
-      unpack_e4m3x2(ws[k] >> 16, f[4 * k + 2], f[4 * k + 3]);
-    }
-  } else if constexpr (Storage<T>::kDtype == ATTN_I8) {
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) f[4 * k + b] = (float)(int8_t)(ws[k] >> (8 * b));
-  } else if constexpr (sizeof(T) == 4) {
+  if constexpr (sizeof(T) == 4) {
     f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
     f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
   } else if constexpr (Storage<T>::kDtype == ATTN_BF16) {

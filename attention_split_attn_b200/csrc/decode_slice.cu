@@ -37,6 +37,7 @@
 #include "decode_tile.cuh"
 #include "internal.h"
 #include "mma.cuh"
+#include "quant.cuh"
 
 namespace attn {
 
@@ -83,7 +84,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   using Geo = DecodeGeom<KT, D>;
   using Sm = DecodeSmem<KT, D, HPW, HG>;
   constexpr int NCW = kKeyWarps * HG;
-  constexpr bool kQuant = Storage<KT>::kDtype == ATTN_FP8_E4M3 || Storage<KT>::kDtype == ATTN_I8;
+  constexpr bool kQuant = is_code_type<KT>();
   constexpr int NS = Geo::NSTAGE;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::kBarOffset);
@@ -238,7 +239,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll
       for (int v = 0; v < Geo::VPL; ++v) {
         const uint4 w = *reinterpret_cast<const uint4*>(sk + j * D + (v * Geo::LPK + dl) * Geo::EPV);
-        unpack_vec<KT>(w, kf + v * Geo::EPV);
+        unpack_kv<KT>(w, kf + v * Geo::EPV);
       }
       float acc[HPW];
 #pragma unroll
@@ -287,7 +288,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int v = 0; v < Geo::VPL; ++v) {
         uint4 w = *reinterpret_cast<const uint4*>(sv + j * D + (v * Geo::LPK + dl) * Geo::EPV);
         if (!vis[i]) w = make_uint4(0u, 0u, 0u, 0u);
-        unpack_vec<KT>(w, vf + v * Geo::EPV);
+        unpack_kv<KT>(w, vf + v * Geo::EPV);
       }
       // quantized cache: p (s_v code) = (p s_v) code
       const float vs = kQuant ? (vis[i] ? __ldg(p.v_scale + (int64_t)(tile0 + j) * p.scale_sc + g) : 0.f) : 1.f;
