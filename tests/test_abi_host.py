@@ -152,6 +152,35 @@ def test_quantized_decode_slice_plan(lib):
     assert ws == (slots * 128 * 4 + 255) // 256 * 256 + (slots * 2 * 4 + 255) // 256 * 256
 
 
+def test_binding_quantized_scale_arguments(lib):
+    """The binding marshals e4m3 caches with their scales and refuses malformed
+    scale tensors before anything reaches the library (CPU tensors: only the
+    argument block is built and validated, nothing is launched)."""
+    import torch
+    q = torch.zeros((2, 8, 128), dtype=torch.bfloat16)
+    out = torch.zeros((2, 8, 128), dtype=torch.bfloat16)
+    k = torch.zeros((64, 2, 128), dtype=torch.uint8).view(torch.float8_e4m3fn)
+    v = torch.zeros((64, 2, 128), dtype=torch.uint8).view(torch.float8_e4m3fn)
+    ks = torch.ones((64, 2), dtype=torch.float32)
+    vs = torch.ones((64, 2), dtype=torch.float32)
+    a = A.make_args(q, k, v, out, scale=0.1, k_scale=ks, v_scale=vs)
+    assert a.kv_type == A.ATTN_FP8_E4M3 and a.scale_stride_cell == 2
+    assert a.k_scale == ks.data_ptr() and a.v_scale == vs.data_ptr()
+    assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == 0
+    assert lib.attn_supports(ctypes.byref(a), A.OP_SELECTED) == -2
+    with pytest.raises(ValueError):
+        A.make_args(q, k, v, out, scale=0.1, k_scale=ks)                      # v_scale missing
+    with pytest.raises(ValueError):
+        A.make_args(q, k, v, out, scale=0.1, k_scale=ks.double(), v_scale=vs)   # not float32
+    with pytest.raises(ValueError):
+        A.make_args(q, k, v, out, scale=0.1, k_scale=ks[:32], v_scale=vs[:32])  # wrong cell count
+    i8 = torch.zeros((64, 2, 128), dtype=torch.int8)
+    a = A.make_args(q, i8, i8.clone(), out, scale=0.1, k_scale=ks, v_scale=vs)
+    assert a.kv_type == A.ATTN_I8
+    a = A.make_args(q, i8, i8.clone(), out, scale=0.1)                          # scales missing
+    assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1
+
+
 def test_strerror(lib):
     for code, name in A.STATUS.items():
         assert lib.attn_strerror(code).decode() == name
