@@ -328,11 +328,16 @@ def random_problem(seed: int, R: int = 3, Hq: int = 4, Hkv: int = 2, D: int = 64
                    seqs: int = 0, causal: bool = False, mask_frac: float = 0.0,
                    softcap: float = 0.0, alibi: bool = False, sinks: bool = False,
                    n_slices: int = 0, scale: Optional[float] = None,
-                   value_scale: float = 1.0) -> Problem:
+                   value_scale: float = 1.0, positions: str = "given",
+                   overhang: int = 0) -> Problem:
     """A small dense-visibility problem.  Each row r gets a range
     [begin_r, begin_r + len_r) inside [0, N) (or the whole cache when
     ranges=False); optional sequence ids, positions, mask, softcap, ALiBi
-    and sinks."""
+    and sinks.  positions (used when causal or alibi): "given" (a random
+    permutation of cell positions and random row positions), "none" (both
+    left unset, so the defaults from the range apply), "row" (row positions
+    only), "cell" (cell positions only).  overhang > 0 moves each range's ends
+    by up to that many cells past 0 and N (a range partly outside the cache)."""
     rng = np.random.default_rng(seed)
     q_dtype = q_dtype or kv_dtype
     q = _normal(rng, (R, Hq, D), F32) * value_scale
@@ -346,14 +351,23 @@ def random_problem(seed: int, R: int = 3, Hq: int = 4, Hkv: int = 2, D: int = 64
         if lengths is None:
             lengths = [int(x) for x in rng.integers(0, N + 1, size=R)]
         begins = [int(rng.integers(0, N - l + 1)) for l in lengths]
+        ends = [b + l for b, l in zip(begins, lengths)]
+        if overhang > 0:
+            begins = [b - int(rng.integers(0, overhang + 1)) if b == 0 or rng.random() < 0.5 else b
+                      for b in begins]
+            ends = [e + int(rng.integers(0, overhang + 1)) if e == N or rng.random() < 0.5 else e
+                    for e in ends]
         p.row_begin = _i32(begins)
-        p.row_end = _i32([b + l for b, l in zip(begins, lengths)])
+        p.row_end = _i32(ends)
     if seqs:
         p.cell_seq = _i32(rng.integers(0, seqs, size=N))
         p.row_seq = _i32(rng.integers(0, seqs, size=R))
     if causal or alibi:
-        p.cell_pos = _i32(rng.permutation(N))
-        p.row_pos = _i32(rng.integers(0, N, size=R))
+        cpos, rpos = rng.permutation(N), rng.integers(0, N, size=R)
+        if positions in ("given", "cell"):
+            p.cell_pos = _i32(cpos)
+        if positions in ("given", "row"):
+            p.row_pos = _i32(rpos)
     if mask_frac > 0:
         m = rng.standard_normal((R, N)).astype(np.float32)
         m[rng.random((R, N)) < mask_frac] = -np.inf

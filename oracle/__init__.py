@@ -36,6 +36,7 @@ MUTATIONS = {
     "empty_row_nan": 5, "gqa_modulo": 6, "no_dedup": 7, "mask_narrowed": 8,
     "invalid_clamped": 9, "scale_after_cap": 10, "neg_inf_mask_added": 11,
     "causal_strict": 12, "seq_ignored": 13, "k_d_reversed": 14,
+    "cell_pos_no_begin": 15, "row_pos_no_minus1": 16, "pos_from_clipped": 17,
     # planted in the dequantization of e4m3 / int8 caches below (Python side)
     "e4m3_bias_8": 101, "e4m3_nan_as_number": 102, "scale_cells_reversed": 103,
     "scale_heads_reversed": 104, "k_scale_for_v": 105, "int8_as_unsigned": 106,

@@ -42,6 +42,9 @@ enum {
     MUT_CAUSAL_STRICT = 12,        /* cell_pos < row_pos (drops the diagonal)  */
     MUT_SEQ_IGNORED = 13,          /* sequence filter not applied              */
     MUT_K_D_REVERSED = 14,         /* score reads k[c,g,D-1-d]                 */
+    MUT_CELL_POS_NO_BEGIN = 15,    /* default cell position c, not c - begin   */
+    MUT_ROW_POS_NO_MINUS1 = 16,    /* default row position end - begin         */
+    MUT_POS_FROM_CLIPPED = 17,     /* default positions from the clipped range */
 };
 
 static int n_online_cores(void) {
@@ -52,17 +55,25 @@ static int n_online_cores(void) {
 /* ---- visibility --------------------------------------------------------- */
 
 static int32_t row_begin_of(const oracle_problem *p, int r) {
-    return p->row_begin ? p->row_begin[r] : 0;
+    int32_t b = p->row_begin ? p->row_begin[r] : 0;
+    if (g_mutation == MUT_POS_FROM_CLIPPED && b < 0) b = 0;
+    return b;
 }
 static int32_t row_end_of(const oracle_problem *p, int r) {
-    return p->row_end ? p->row_end[r] : p->n_cells;
+    int32_t e = p->row_end ? p->row_end[r] : p->n_cells;
+    if (g_mutation == MUT_POS_FROM_CLIPPED && e > p->n_cells) e = p->n_cells;
+    return e;
 }
+/* Default positions (cell c at c - begin, the row at end - begin - 1) come
+ * from the range as the caller gave it; only visibility clips it to the cache. */
 static int64_t row_pos_of(const oracle_problem *p, int r) {
     if (p->row_pos) return p->row_pos[r];
+    if (g_mutation == MUT_ROW_POS_NO_MINUS1) return (int64_t)row_end_of(p, r) - row_begin_of(p, r);
     return (int64_t)row_end_of(p, r) - row_begin_of(p, r) - 1;
 }
 static int64_t cell_pos_of(const oracle_problem *p, int r, int32_t c) {
     if (p->cell_pos) return p->cell_pos[c];
+    if (g_mutation == MUT_CELL_POS_NO_BEGIN) return (int64_t)c;
     return (int64_t)c - row_begin_of(p, r);
 }
 

@@ -38,12 +38,15 @@
  *    must not depend on another's cells): same page, "Isolation" measurements.
  *  - the FP64 reference compared by NMSE: same page, #119 commit message.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - GQA mapping g = floor(h / G); ALiBi bias = -slope_h * |row_pos - cell_pos|;
  *  - a mask value of exactly -inf excludes the cell (it is never read); any
  *    other value (finite, +inf, NaN) is added;
  *  - the sink is one extra logit with no value vector, applied raw;
- *  - selection entries < 0 or >= n_cells are invalid; duplicates count once.
+ *  - selection entries < 0 or >= n_cells are invalid; duplicates count once;
+ *  - with no explicit positions, cell c sits at c - row_begin and the row at
+ *    row_end - row_begin - 1, from the range as given (a range reaching outside
+ *    [0, n_cells) is clipped for visibility only).
  */
 #ifndef ATTN_ORACLE_H
 #define ATTN_ORACLE_H

@@ -71,6 +71,23 @@ def _close(a, b, rtol=1e-13, atol=1e-300):
 # Library reference: torch SDPA in float64
 # ----------------------------------------------------------------------------
 
+def _positions(p):
+    """Cell positions per row [R, N] and row positions [R] (int64).  Where the
+    problem gives none, the boundary's defaults (the C ABI's "Positions"
+    rule): cell c of row r sits at c - row_begin[r] and row r at
+    row_end[r] - row_begin[r] - 1, from the range as given, even where it
+    reaches outside [0, N)."""
+    R, N = p.n_rows, p.n_cells
+    b = p.row_begin.numpy().astype(np.int64) if p.row_begin is not None else np.zeros(R, np.int64)
+    e = p.row_end.numpy().astype(np.int64) if p.row_end is not None else np.full(R, N, np.int64)
+    if p.cell_pos is not None:
+        cpos = np.broadcast_to(p.cell_pos.numpy().astype(np.int64)[None, :], (R, N))
+    else:
+        cpos = np.arange(N, dtype=np.int64)[None, :] - b[:, None]
+    rpos = p.row_pos.numpy().astype(np.int64) if p.row_pos is not None else e - b - 1
+    return cpos, rpos
+
+
 def _visibility_bias(p):
     """[Hq, R, N] float64 bias: -inf where invisible, mask + textbook ALiBi where visible."""
     R, Hq, N = p.n_rows, p.n_head_q, p.n_cells
@@ -82,10 +99,9 @@ def _visibility_bias(p):
         vis &= (cols[None, :] >= b) & (cols[None, :] < e)
     if p.cell_seq is not None and p.row_seq is not None:
         vis &= p.cell_seq.numpy()[None, :] == p.row_seq.numpy()[:, None]
-    cpos = p.cell_pos.numpy().astype(np.int64) if p.cell_pos is not None else None
-    rpos = p.row_pos.numpy().astype(np.int64) if p.row_pos is not None else None
+    cpos, rpos = _positions(p)
     if p.causal:
-        vis &= cpos[None, :] <= rpos[:, None]
+        vis &= cpos <= rpos[:, None]
     bias = np.zeros((Hq, R, N), dtype=np.float64)
     if p.mask is not None:
         m = p.mask.numpy().astype(np.float64)
@@ -94,7 +110,7 @@ def _visibility_bias(p):
     if p.alibi_slopes is not None:
         # textbook causal ALiBi (Press et al.): bias = slope * (j - i) for key j <= query i
         assert p.causal, "the library pin covers causal ALiBi only"
-        rel = (cpos[None, :] - rpos[:, None]).astype(np.float64)       # <= 0 where visible
+        rel = (cpos - rpos[:, None]).astype(np.float64)                # <= 0 where visible
         slopes = p.alibi_slopes.numpy().astype(np.float64)
         bias += slopes[:, None, None] * np.where(vis, rel, 0.0)[None]
     bias[:, ~vis] = -INF
@@ -152,6 +168,17 @@ def pin_sdpa_alibi_textbook():
     for seed in range(4):
         _compare_with_sdpa(W.random_problem(200 + seed, R=5, Hq=4, Hkv=1, D=8, N=50,
                                             ranges=False, causal=True, alibi=True))
+
+
+def pin_sdpa_default_positions():
+    """No cell and/or row positions given: the defaults come from each row's
+    range as given (nonzero and negative begins, ends past N), under causality,
+    ALiBi and sinks."""
+    for seed in range(4):
+        for mode in ("none", "row", "cell"):
+            _compare_with_sdpa(W.random_problem(400 + seed, R=7, Hq=4, Hkv=2, D=8, N=40,
+                                                causal=True, alibi=True, sinks=True,
+                                                positions=mode, overhang=6 * (seed % 2)))
 
 
 def pin_sdpa_sinks():
