@@ -67,24 +67,32 @@ __device__ int g_status_word = 0;
 namespace attn {
 namespace {
 
+// A failed runtime query is cleared (cudaGetLastError) before returning, so
+// that a later launch check does not report it again.
 int32_t device_info(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
     return fail(ATTN_ERR_CUDA, "cudaGetDevice failed");
+  }
   std::lock_guard<std::mutex> lk(g_dev_mutex);
   DeviceInfo& d = g_dev[dev];
   if (!d.init) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
       return fail(ATTN_ERR_CUDA, "cannot query device %d", dev);
+    }
     if (major != 10 || minor != 0)
       return fail(ATTN_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
                   major, minor);
     void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess)
+    if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) {
+      cudaGetLastError();
       return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    }
     d.status = static_cast<int*>(addr);
     d.init = true;
   }
@@ -483,6 +491,10 @@ int32_t run_unified(const attn_args* a, void* ws, size_t ws_bytes, cudaStream_t 
 
 namespace attn {
 void set_last_error(const char* msg) { g_last_error = msg; }
+int32_t check_device() {
+  DeviceInfo* di = nullptr;
+  return device_info(&di);
+}
 }  // namespace attn
 
 using namespace attn;

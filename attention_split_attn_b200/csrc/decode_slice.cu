@@ -104,10 +104,11 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     r = (int)(bid / ((int64_t)p.S * p.Hkv));
   }
   RowCtx rc;
-  rc.begin = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
-  rc.end = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
-  rc.begin = max(rc.begin, 0);
-  rc.end = min(rc.end, p.N);
+  const int32_t raw_b = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
+  const int32_t raw_e = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
+  rc.pos_base = raw_b;
+  rc.begin = max(raw_b, 0);
+  rc.end = min(raw_e, p.N);
   if (rc.end < rc.begin) rc.end = rc.begin;
   {
     const int64_t b = rc.begin, e = rc.end;
@@ -124,7 +125,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     return;
   }
   rc.row_seq = p.f.row_seq ? __ldg(p.f.row_seq + r) : 0;
-  rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + r) : (int64_t)(rc.end - rc.begin - 1);
+  rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + r) : (int64_t)raw_e - raw_b - 1;
   const bool has_filter = (p.f.cell_seq && p.f.row_seq) || p.f.causal || p.f.mask;
   const int n_tiles = (rc.s_end - rc.s_begin + kTileKeys - 1) / kTileKeys;
 
@@ -231,7 +232,7 @@ decode_slice_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       const int c = tile0 + j;
       bool vk = c < rc.s_end;
       float mval = 0.f;
-      int64_t cpos = c - rc.begin;
+      int64_t cpos = (int64_t)c - rc.pos_base;
       if (has_filter && vk) vk = cell_visible(p.f, rc, r, c, mval, cpos);
       else if (alibi && p.f.cell_pos && vk) cpos = __ldg(p.f.cell_pos + c);
       vis[i] = vk;
@@ -387,10 +388,11 @@ decode_warp_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     r = (int)(bid / ((int64_t)p.S * p.Hkv));
   }
   RowCtx rc;
-  rc.begin = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
-  rc.end = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
-  rc.begin = max(rc.begin, 0);
-  rc.end = min(rc.end, p.N);
+  const int32_t raw_b = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
+  const int32_t raw_e = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
+  rc.pos_base = raw_b;
+  rc.begin = max(raw_b, 0);
+  rc.end = min(raw_e, p.N);
   if (rc.end < rc.begin) rc.end = rc.begin;
   {
     const int64_t b = rc.begin, e = rc.end;
@@ -404,7 +406,7 @@ decode_warp_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     return;
   }
   rc.row_seq = p.f.row_seq ? __ldg(p.f.row_seq + r) : 0;
-  rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + r) : (int64_t)(rc.end - rc.begin - 1);
+  rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + r) : (int64_t)raw_e - raw_b - 1;
   const bool has_filter = (p.f.cell_seq && p.f.row_seq) || p.f.causal || p.f.mask;
   const int n_tiles = (rc.s_end - rc.s_begin + kWarpTile - 1) / kWarpTile;
 

@@ -91,13 +91,16 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodePlan p) {
 struct Cursor {
   int r, g;
   int64_t j, nt;
-  int32_t begin, end;
+  int32_t begin, end;        // the row's cell range, clipped to [0, n_cells)
+  int32_t raw_b, raw_e;      // row_begin / row_end as given (default positions)
 };
 
 __device__ __forceinline__ void cursor_load_row(const DecodePlan& p, const int64_t* row_tiles, Cursor& c) {
   c.nt = row_tiles[c.r + 1] - row_tiles[c.r];
   int32_t b = p.f.row_begin ? __ldg(p.f.row_begin + c.r) : 0;
   int32_t e = p.f.row_end ? __ldg(p.f.row_end + c.r) : p.N;
+  c.raw_b = b;
+  c.raw_e = e;
   b = max(b, 0);
   e = min(e, p.N);
   c.begin = b;
@@ -207,10 +210,11 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     RowCtx rc;
     rc.begin = cc.begin;
     rc.end = cc.end;
+    rc.pos_base = cc.raw_b;
     rc.s_begin = cc.begin;
     rc.s_end = cc.end;
     rc.row_seq = p.f.row_seq ? __ldg(p.f.row_seq + cc.r) : 0;
-    rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + cc.r) : (int64_t)(cc.end - cc.begin - 1);
+    rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + cc.r) : (int64_t)cc.raw_e - cc.raw_b - 1;
     return rc;
   };
   RowCtx rc = make_ctx(c);

@@ -23,7 +23,8 @@ namespace attn {
 constexpr int kWarpTile = 16;   // cells per warp tile = one MMA m-tile
 
 struct RowCtx {
-  int32_t begin, end;        // the row's cell range
+  int32_t begin, end;        // the row's cell range, clipped to [0, n_cells)
+  int32_t pos_base;          // row_begin as given (not clipped): cell c's default position is c - pos_base
   int32_t s_begin, s_end;    // the cells this unit may use
   int32_t row_seq;
   int64_t row_pos;
@@ -33,7 +34,7 @@ __device__ __forceinline__ bool cell_visible(const RowFilter& f, const RowCtx& r
                                              float& mval, int64_t& cpos) {
   bool vis = true;
   if (f.cell_seq != nullptr && f.row_seq != nullptr) vis = (__ldg(f.cell_seq + c) == rc.row_seq);
-  cpos = f.cell_pos ? (int64_t)__ldg(f.cell_pos + c) : (int64_t)(c - rc.begin);
+  cpos = f.cell_pos ? (int64_t)__ldg(f.cell_pos + c) : (int64_t)c - rc.pos_base;
   if (f.causal) vis = vis && (cpos <= rc.row_pos);
   mval = 0.f;
   if (f.mask != nullptr) {
@@ -178,7 +179,7 @@ struct WarpTileState {
       float mval = 0.f;
       float negdist = 0.f;
       if (has_filter || alibi) {
-        int64_t cpos = c - rc.begin;
+        int64_t cpos = (int64_t)c - rc.pos_base;
         if (has_filter && vk) vk = cell_visible(p.f, rc, r, c, mval, cpos);
         else if (alibi && p.f.cell_pos && vk) cpos = __ldg(p.f.cell_pos + c);
         negdist = -(float)(rc.row_pos >= cpos ? rc.row_pos - cpos : cpos - rc.row_pos);

@@ -194,4 +194,8 @@ int max_tree_rows();
 // Set the message attn_last_error() returns on this thread.
 void set_last_error(const char* msg);
 
+// ATTN_OK when the current device is one the kernels run on (sm_100), else
+// the status the operations return for it (with attn_last_error() set).
+int32_t check_device();
+
 }  // namespace attn

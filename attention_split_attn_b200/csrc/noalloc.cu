@@ -48,8 +48,15 @@ void* g_scratch_ptr[kMaxDevices] = {};
 }  // namespace
 
 extern "C" int32_t attn_decode_noalloc(const attn_args* args, void* stream) {
+  // Arguments and device first, so this call refuses exactly what attn_decode
+  // refuses (an unsupported device included) before touching the array.
+  const int32_t ok = attn_supports(args, ATTN_OP_DECODE);
+  if (ok != ATTN_OK) return ok;
+  const int32_t dev_ok = attn::check_device();
+  if (dev_ok != ATTN_OK) return dev_ok;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();   // leave no error behind for the next call to report
     attn::set_last_error("attn_decode_noalloc: no usable current device");
     return ATTN_ERR_CUDA;
   }
@@ -60,6 +67,7 @@ extern "C" int32_t attn_decode_noalloc(const attn_args* args, void* stream) {
       void* p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
         attn::set_last_error("attn_decode_noalloc: cudaGetSymbolAddress of the scratch array failed");
         return ATTN_ERR_CUDA;
       }
@@ -67,8 +75,6 @@ extern "C" int32_t attn_decode_noalloc(const attn_args* args, void* stream) {
     }
     scratch = g_scratch_ptr[dev];
   }
-  const int32_t ok = attn_supports(args, ATTN_OP_DECODE);
-  if (ok != ATTN_OK) return ok;
   const size_t need = attn_workspace_size(args, ATTN_OP_DECODE, 0);
   if (need > kNoAllocScratchBytes) {
     char msg[256];

@@ -555,12 +555,13 @@ __global__ void __launch_bounds__(kVisThreads) visible_list_kernel(const Selecte
   __shared__ int wcount[32];
   __shared__ int base_sh;
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  int32_t rb = f.row_begin ? __ldg(f.row_begin + r) : 0;
-  int32_t re = f.row_end ? __ldg(f.row_end + r) : p.N;
-  rb = max(rb, 0);
-  re = min(re, p.N);
+  // positions default from the range as given; the scan covers its part inside [0, n_cells)
+  const int32_t raw_b = f.row_begin ? __ldg(f.row_begin + r) : 0;
+  const int32_t raw_e = f.row_end ? __ldg(f.row_end + r) : p.N;
+  const int32_t rb = max(raw_b, 0);
+  const int32_t re = min(raw_e, p.N);
   const int32_t rs = f.row_seq ? __ldg(f.row_seq + r) : 0;
-  const int32_t rp = f.row_pos ? __ldg(f.row_pos + r) : re - rb - 1;
+  const int64_t rp = f.row_pos ? (int64_t)__ldg(f.row_pos + r) : (int64_t)raw_e - raw_b - 1;
   const float* mrow = f.mask ? f.mask + (int64_t)r * f.mask_sr : nullptr;
   int32_t* out = p.compact + (int64_t)r * p.n_sel;
   if (tid == 0) base_sh = 0;
@@ -573,7 +574,7 @@ __global__ void __launch_bounds__(kVisThreads) visible_list_kernel(const Selecte
       bool v = c < re;
       if (v && f.cell_seq) v = __ldg(f.cell_seq + c) == rs;
       if (v && f.causal) {
-        const int32_t cp = f.cell_pos ? __ldg(f.cell_pos + c) : (int32_t)(c - rb);
+        const int64_t cp = f.cell_pos ? (int64_t)__ldg(f.cell_pos + c) : c - raw_b;
         v = cp <= rp;
       }
       if (v && mrow) v = !(__ldg(mrow + c) == neg_inf());

@@ -13,7 +13,8 @@
 // One CTA per row: the row walks its parent chain into a shared-memory bitmap
 // of tree nodes (at most n_rows steps: a parent index that is not smaller than
 // its child, or out of range, ends the walk and records ATTN_ERR_INVALID_ARG in
-// the device status word, leaving the row's tree cells hidden), then writes
+// the device status word; the nodes walked up to that link, the row itself
+// included, stay visible and the ancestors above it are hidden), then writes
 // the mask row with coalesced stores.
 #include "common.cuh"
 #include "internal.h"

@@ -60,8 +60,11 @@
  *   and cell_pos[c] <= row_pos[r]             (if causal)
  *   and mask[r, c] != -inf                    (if mask; a -inf cell is never read)
  * Positions: cell_pos NULL -> c - row_begin[r]; row_pos NULL ->
- * row_end[r] - row_begin[r] - 1.  Selected: the distinct entries e of row r's
- * list with 0 <= e < n_cells; no range, sequence, causal or mask filter.
+ * row_end[r] - row_begin[r] - 1, both from row_begin/row_end as given: a
+ * range reaching below 0 or past n_cells is clipped to [0, n_cells) for
+ * visibility only, never for positions.  Selected: the distinct entries e of
+ * row r's list with 0 <= e < n_cells; no range, sequence, causal or mask
+ * filter.
  *
  * Memory and ownership.  Every pointer in the argument blocks is DEVICE
  * memory owned by the caller.  The caller also owns the workspace (sized by

@@ -65,6 +65,18 @@ def poisoned_workspace(nbytes, device="cuda"):
     return torch.full((nbytes,), 0xFF, dtype=torch.uint8, device=device)
 
 
+def run_prefill(p, **over):
+    (q, k, v, out), kw = A.problem_kwargs(p)
+    kw.update(over)
+    out.fill_(float("nan"))
+    args = A.make_args(q, k, v, out, **kw)
+    ws = poisoned_workspace(A.workspace_size(args, A.OP_PREFILL))
+    A.attn_prefill_args(args, ws=ws)
+    torch.cuda.synchronize()
+    A.check_device_status()
+    return out
+
+
 def run_decode(p, **over):
     (q, k, v, out), kw = A.problem_kwargs(p)
     kw.update(over)

@@ -77,6 +77,18 @@ def test_boundary_lengths(cuda_lib, length):
         check(p, run_decode(p, n_slices=S, max_row_len=length), f"len={length} S={S}", ref=ref)
 
 
+@pytest.mark.parametrize("kv", [torch.float32, torch.bfloat16])
+def test_max_row_len_below_real_length(cuda_lib, kv):
+    """max_row_len only sizes the slices: rows longer than it are still
+    computed in full, the last slice taking the excess."""
+    p = W.random_problem(77 + (kv == torch.bfloat16), R=5, Hq=8, Hkv=2, D=128, N=2000, kv_dtype=kv,
+                         out_dtype=torch.float32, lengths=[2000, 1500, 700, 90, 0], sinks=True)
+    ref = oracle.attn(p)
+    for S in (0, 2, 5, 17, 64):
+        for mrl in (1, 33, 100, 999):
+            check(p, run_decode(p, n_slices=S, max_row_len=mrl), f"S={S} max_row_len={mrl}", ref=ref)
+
+
 def test_launch_guard_16_rows_over_33_keys(cuda_lib):
     """TensorFold PR #2595's planted control went red at 16 rows over 33 keys
     with more slices than rows; here every slice count must stay inside the

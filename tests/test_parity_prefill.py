@@ -21,21 +21,9 @@ import torch
 import oracle
 import attention_split_attn_b200 as A
 from attention_split_attn_b200 import workloads as W
-from parity import check, poisoned_workspace
+from parity import check, poisoned_workspace, run_prefill
 
 pytestmark = pytest.mark.gpu
-
-
-def run_prefill(p, **over):
-    (q, k, v, out), kw = A.problem_kwargs(p)
-    kw.update(over)
-    out.fill_(float("nan"))
-    args = A.make_args(q, k, v, out, **kw)
-    ws = poisoned_workspace(A.workspace_size(args, A.OP_PREFILL))
-    A.attn_prefill_args(args, ws=ws)
-    torch.cuda.synchronize()
-    A.check_device_status()
-    return out
 
 
 @pytest.mark.parametrize("kv", [torch.float16, torch.bfloat16])

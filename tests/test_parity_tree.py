@@ -73,12 +73,20 @@ def test_tree_decode_full_heads_orders_bit_identical(cuda_lib):
 
 def test_tree_mask_rejects_a_parent_that_is_not_smaller(cuda_lib):
     """A parent index >= its child is not heap order: the kernel's own check
-    stops the walk and the device status word reports it."""
+    stops the walk and the device status word reports it.  The nodes walked
+    up to the bad link (the row itself included) stay visible; the ancestors
+    above it are hidden."""
     p = W.tree_decode(width=8, visible=100, Hq=4, Hkv=1, D=64)
     parent = p.tree_parent.clone()
     parent[5] = 6
-    A.tree_mask(parent.cuda(), p.tree_prefix, p.n_cells)
+    mask = A.tree_mask(parent.cuda(), p.tree_prefix, p.n_cells)
     with pytest.raises(A.AttnError) as e:
         A.check_device_status()
     assert e.value.status == -1
     A.check_device_status()   # the status word was cleared
+    row5 = mask[5].cpu()
+    assert torch.all(row5[:p.tree_prefix] == 0)
+    tree = row5[p.tree_prefix:p.tree_prefix + p.n_rows]
+    expect = torch.full_like(tree, float("-inf"))
+    expect[5] = 0.0
+    assert torch.equal(tree, expect)
