@@ -19,6 +19,7 @@
 #include <string>
 
 #include "attn.h"
+#include "common.cuh"
 #include "internal.h"
 
 namespace attn {
@@ -159,7 +160,7 @@ bool is_quantized(int32_t t) { return t == ATTN_FP8_E4M3 || t == ATTN_I8; }
 
 int32_t validate_common(const attn_args* a, int32_t op) {
   if (!a) return fail(ATTN_ERR_INVALID_ARG, "args is NULL");
-  for (int i = 0; i < 5; ++i)
+  for (int i = op == ATTN_OP_PREFILL ? 1 : 0; i < 5; ++i)
     if (a->reserved[i] != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved fields must be zero");
   if (a->n_rows < 0 || a->n_cells < 0) return fail(ATTN_ERR_INVALID_ARG, "negative n_rows or n_cells");
   if (a->n_head_q <= 0 || a->n_head_kv <= 0)
@@ -357,6 +358,8 @@ SelWs selected_ws_layout(const attn_args* a, int n_sel, const SelShape& sh) {
 // ---- prefill planning ---------------------------------------------------------------
 constexpr int kPfTile = 128;   // rows and cells per prefill tile
 
+bool unified_route(const attn_args* a);
+
 int32_t check_prefill(const attn_args* a) {
   int32_t st = validate_common(a, ATTN_OP_PREFILL);
   if (st != ATTN_OK) return st;
@@ -365,6 +368,10 @@ int32_t check_prefill(const attn_args* a) {
   if (a->q_type != a->kv_type) return fail(ATTN_ERR_UNSUPPORTED, "prefill: Q must be in the K/V dtype");
   if (a->head_dim != 64 && a->head_dim != 128)
     return fail(ATTN_ERR_UNSUPPORTED, "prefill: head_dim %d not in {64, 128}", a->head_dim);
+  if (a->reserved[0] < 0 || a->reserved[0] > 1000000)
+    return fail(ATTN_ERR_INVALID_ARG, "prefill: reserved[0] (the bounded-wait test) must be 0..1000000 us");
+  if (a->reserved[0] != 0 && unified_route(a))
+    return fail(ATTN_ERR_INVALID_ARG, "prefill: the bounded-wait test runs on the dense tensor-core kernel only");
   if (a->n_rows > 0) {
     if (!aligned16(a->q)) return fail(ATTN_ERR_UNSUPPORTED, "prefill: q must be 16-byte aligned");
     if ((a->n_rows > 1 && (a->q_stride_row % 8)) || (a->n_head_q > 1 && (a->q_stride_head % 8)) ||
@@ -780,6 +787,8 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
               (a->n_head_q <= 1 || a->o_stride_head % ovec == 0);
   p.mask_vec = a->mask && aligned16(a->mask) && (a->n_rows <= 1 || a->mask_stride_row % 4 == 0);
   p.status = di->status;
+  p.wait_ns = a->reserved[0] > 0 ? (uint64_t)a->reserved[0] * 1000ull : kWaitLimitNs;
+  p.test_stall = a->reserved[0] > 0 ? 1 : 0;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   record_event(events, 0, s);

@@ -163,6 +163,8 @@ struct PrefillPlan {
   int32_t out_vec;          // output rows may be written with 16-byte stores
   int32_t mask_vec;         // mask rows may be read with 16-byte loads
   int* status;
+  uint64_t wait_ns;         // bound of every barrier wait (a timeout records ATTN_ERR_DEVICE_TIMEOUT)
+  int32_t test_stall;       // 1: the softmax warps first wait on a barrier nothing arrives at
 };
 
 cudaError_t launch_prefill(const PrefillPlan& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,

@@ -75,44 +75,96 @@ __device__ __forceinline__ RowVis row_vis(const RowFilter& f, int r, int N) {
   return v;
 }
 
-// Block (rt, kt) for blockIdx.x < n_rt * n_kt; block (kt, g) of the V scan
-// after that.  256 threads; thread t looks at cell t % 128 of the tile and
-// at rows t / 128, t / 128 + 2, ...
-__global__ void __launch_bounds__(256) prefill_classify_kernel(PrefillPlan p) {
+// Blocks (rt, kt) for blockIdx.x < n_rt * n_kt classify one tile each; blocks
+// (kt, g) after them scan one cell tile of one KV head.  256 threads.
+//  * Classification: the 128 rows' range, sequence and position are staged in
+//    shared memory; warp w takes rows w, w + 8, ..., lane l cells 4l .. 4l + 3
+//    of the tile, and with a mask each warp issues its 16 rows' 16-byte mask
+//    loads before using any of them (the scan is bound by DRAM latency
+//    otherwise).  A row's visibility bits are gathered from the lanes' nibbles
+//    by three shuffles per 8-lane group (word k = cells 32k .. 32k + 31).
+//  * V scan and K norms: every 16-byte chunk of the tile's V and K rows of
+//    head g is loaded before any is used.
+constexpr int kClsThreads = 256;
+constexpr int kClsRowsPerWarp = kPfRows / (kClsThreads / 32);   // 16
+
+__global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPlan p) {
   pdl_launch_dependents();   // the prefill kernel may start its prologue
-  const int tid = threadIdx.x;
+  __shared__ int4 rows_sh[kPfRows];
+  __shared__ float wmax[kClsThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t b = blockIdx.x;
   const int64_t n_cls = (int64_t)p.n_rt * p.n_kt;
   if (b < n_cls) {
     const int rt = (int)(b / p.n_kt), kt = (int)(b % p.n_kt);
-    const int c = kt * kPfCells + (tid & 127);
-    const bool cin = c < p.N;
-    const int32_t cs = (cin && p.f.cell_seq) ? __ldg(p.f.cell_seq + c) : 0;
-    const int32_t cpos_given = (cin && p.f.cell_pos) ? __ldg(p.f.cell_pos + c) : 0;
-    bool any = false, notfull = false, bias = false, late = false;
-    const int r_end = min(p.R, (rt + 1) * kPfRows);
-    // every warp walks the same rows (its 32 cells of one row per step), so
-    // its ballot is one 32-bit word of that row's visibility bits
-    for (int r = rt * kPfRows + (tid >> 7); r < r_end; r += 2) {
-      const RowVis rv = row_vis(p.f, r, p.N);
-      bool vis = cin && c >= rv.rb && c < rv.re;
-      if (p.f.cell_seq) vis = vis && cs == rv.rs;
-      const int32_t cp = p.f.cell_pos ? cpos_given : c - rv.rb;
-      if (p.f.causal) vis = vis && cp <= rv.rp;
-      bool zero_bias = true;
-      if (p.f.mask && vis) {
-        const float mv = __ldg(p.f.mask + (int64_t)r * p.f.mask_sr + c);
-        vis = !(mv == neg_inf());
-        zero_bias = (mv == 0.f);
+    if (tid < kPfRows) {
+      const int r = rt * kPfRows + tid;
+      const RowVis rv = r < p.R ? row_vis(p.f, r, p.N) : RowVis{0, 0, 0, 0};
+      rows_sh[tid] = make_int4(rv.rb, rv.re, rv.rs, rv.rp);
+    }
+    const int c_base = kt * kPfCells + 4 * lane;
+    bool cin[4];
+    int32_t cs[4], cpg[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = c_base + e;
+      cin[e] = c < p.N;
+      cs[e] = (cin[e] && p.f.cell_seq) ? __ldg(p.f.cell_seq + c) : 0;
+      cpg[e] = (cin[e] && p.f.cell_pos) ? __ldg(p.f.cell_pos + c) : 0;
+    }
+    float4 mv[kClsRowsPerWarp];
+    if (p.f.mask) {
+      const bool vec = p.mask_vec && kt * kPfCells + kPfCells <= p.N;
+#pragma unroll
+      for (int i = 0; i < kClsRowsPerWarp; ++i) {
+        const int r = rt * kPfRows + warp + 8 * i;
+        mv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < p.R) {
+          const float* mrow = p.f.mask + (int64_t)r * p.f.mask_sr + c_base;
+          if (vec) {
+            mv[i] = __ldg(reinterpret_cast<const float4*>(mrow));
+          } else {
+            if (cin[0]) mv[i].x = __ldg(mrow);
+            if (cin[1]) mv[i].y = __ldg(mrow + 1);
+            if (cin[2]) mv[i].z = __ldg(mrow + 2);
+            if (cin[3]) mv[i].w = __ldg(mrow + 3);
+          }
+        }
       }
-      any |= vis;
-      notfull |= !(vis && zero_bias);
-      bias |= vis && !zero_bias;
-      late |= vis && cp > rv.rp;
+    }
+    __syncthreads();
+    bool any = false, notfull = false, bias = false, late = false;
+#pragma unroll
+    for (int i = 0; i < kClsRowsPerWarp; ++i) {
+      const int rl = warp + 8 * i;
+      if (rt * kPfRows + rl >= p.R) continue;   // warp-uniform
+      const int4 rv = rows_sh[rl];
+      const float mvals[4] = {mv[i].x, mv[i].y, mv[i].z, mv[i].w};
+      uint32_t nib = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = c_base + e;
+        bool vis = cin[e] && c >= rv.x && c < rv.y;
+        if (p.f.cell_seq) vis = vis && cs[e] == rv.z;
+        const int32_t cp = p.f.cell_pos ? cpg[e] : c - rv.x;
+        if (p.f.causal) vis = vis && cp <= rv.w;
+        bool zero_bias = true;
+        if (p.f.mask && vis) {
+          vis = !(mvals[e] == neg_inf());
+          zero_bias = (mvals[e] == 0.f);
+        }
+        any |= vis;
+        notfull |= !(vis && zero_bias);
+        bias |= vis && !zero_bias;
+        late |= vis && cp > rv.w;
+        nib |= (vis ? 1u : 0u) << e;
+      }
       if (p.bits) {
-        const uint32_t word = __ballot_sync(0xffffffffu, vis);
-        if ((tid & 31) == 0)
-          p.bits[((b * kPfRows + (r - rt * kPfRows)) << 2) + ((tid & 127) >> 5)] = word;
+        uint32_t word = nib << (4 * (lane & 7));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        word |= __shfl_xor_sync(0xffffffffu, word, 4);
+        if ((lane & 7) == 0) p.bits[((b * kPfRows + rl) << 2) + (lane >> 3)] = word;
       }
     }
     const int a = __syncthreads_or(any ? 1 : 0);
@@ -126,59 +178,67 @@ __global__ void __launch_bounds__(256) prefill_classify_kernel(PrefillPlan p) {
   } else {
     const int64_t vb = b - n_cls;
     const int kt = (int)(vb / p.Hkv), g = (int)(vb % p.Hkv);
-    // 16-byte chunks of the tile's V rows of head g: 128 cells x D/8 chunks.
-    // A 16-bit value is non-finite iff its exponent field is all ones.
+    // 16-byte chunks of the tile's rows of head g: 128 cells x D/8 chunks,
+    // chunk i of this thread = tid + 256 i (per_row chunks of one cell sit in
+    // per_row consecutive lanes; per_row divides 32).
     const int per_row = p.D / 8;
+    const int n_chunk = kPfCells * per_row;
+    constexpr int kMaxPer = kPfCells * 16 / kClsThreads;   // D <= 128
+    const uint16_t* vbase = static_cast<const uint16_t*>(p.v) + (int64_t)g * p.kv_sh;
+    const uint16_t* kbase = static_cast<const uint16_t*>(p.k) + (int64_t)g * p.kv_sh;
+    uint4 vw[kMaxPer], kw[kMaxPer];
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+      const int i = tid + k * kClsThreads;
+      const int c = kt * kPfCells + i / per_row;
+      vw[k] = make_uint4(0u, 0u, 0u, 0u);
+      kw[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < n_chunk && c < p.N) {
+        vw[k] = __ldg(reinterpret_cast<const uint4*>(vbase + (int64_t)c * p.kv_sc) + (i % per_row));
+        if (p.kn2) kw[k] = __ldg(reinterpret_cast<const uint4*>(kbase + (int64_t)c * p.kv_sc) + (i % per_row));
+      }
+    }
+    // A 16-bit value is non-finite iff its exponent field is all ones.
     const uint32_t e_lo = p.kv_type == ATTN_BF16 ? 0x7F80u : 0x7C00u;
     bool bad = false;
-    for (int i = tid; i < kPfCells * per_row; i += 256) {
-      const int c = kt * kPfCells + i / per_row;
-      if (c >= p.N) continue;
-      const uint16_t* row = static_cast<const uint16_t*>(p.v) + (int64_t)c * p.kv_sc + (int64_t)g * p.kv_sh;
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + (i % per_row));
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        bad |= ((ws[k] & e_lo) == e_lo) | (((ws[k] >> 16) & e_lo) == e_lo);
+    for (int k = 0; k < kMaxPer; ++k) {
+      const uint32_t ws[4] = {vw[k].x, vw[k].y, vw[k].z, vw[k].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) bad |= ((ws[q] & e_lo) == e_lo) | (((ws[q] >> 16) & e_lo) == e_lo);
     }
     const int any_bad = __syncthreads_or(bad ? 1 : 0);
     if (tid == 0) p.vbad[(int64_t)kt * p.Hkv + g] = any_bad ? 1 : 0;
     if (p.kn2) {
       // max over the tile's cells of |k_c|^2 (NaN-propagating: a non-finite K
-      // makes the bound fail).  The per_row chunks of one cell sit in
-      // per_row consecutive lanes (per_row divides 32 and 256).
-      __shared__ float wmax[8];
+      // makes the bound fail)
       float mx = 0.f;
-      for (int i = tid; i < kPfCells * per_row; i += 256) {
-        const int c = kt * kPfCells + i / per_row;
-        float ss = 0.f;
-        if (c < p.N) {
-          const uint16_t* row = static_cast<const uint16_t*>(p.k) + (int64_t)c * p.kv_sc + (int64_t)g * p.kv_sh;
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + (i % per_row));
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float lo, hi;
-            if (p.kv_type == ATTN_BF16) {
-              lo = __uint_as_float(ws[k] << 16);
-              hi = __uint_as_float(ws[k] & 0xffff0000u);
-            } else {
-              lo = __half2float(__ushort_as_half((unsigned short)(ws[k] & 0xffffu)));
-              hi = __half2float(__ushort_as_half((unsigned short)(ws[k] >> 16)));
-            }
-            ss = fmaf(lo, lo, ss);
-            ss = fmaf(hi, hi, ss);
+      for (int k = 0; k < kMaxPer; ++k) {
+        const uint32_t ws[4] = {kw[k].x, kw[k].y, kw[k].z, kw[k].w};
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float lo, hi;
+          if (p.kv_type == ATTN_BF16) {
+            lo = __uint_as_float(ws[q] << 16);
+            hi = __uint_as_float(ws[q] & 0xffff0000u);
+          } else {
+            lo = __half2float(__ushort_as_half((unsigned short)(ws[q] & 0xffffu)));
+            hi = __half2float(__ushort_as_half((unsigned short)(ws[q] >> 16)));
           }
+          ss = fmaf(lo, lo, ss);
+          ss = fmaf(hi, hi, ss);
         }
         for (int o = per_row / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         mx = fmax_nan(mx, ss);
       }
       for (int o = 16; o > 0; o >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if ((tid & 31) == 0) wmax[tid >> 5] = mx;
+      if (lane == 0) wmax[warp] = mx;
       __syncthreads();
       if (tid == 0) {
         float m = wmax[0];
-        for (int w8 = 1; w8 < 8; ++w8) m = fmax_nan(m, wmax[w8]);
+        for (int w8 = 1; w8 < kClsThreads / 32; ++w8) m = fmax_nan(m, wmax[w8]);
         p.kn2[(int64_t)kt * p.Hkv + g] = m;
       }
     }
@@ -193,14 +253,15 @@ template <int D>
 struct PfLayout {
   static constexpr int BOX = 128 * 128;                  // one TMA box: 128 rows x 128 B (64 values)
   static constexpr int TILE = kPfRows * D * 2;           // a Q, K or V tile: D/64 boxes
-  static constexpr int PTILE = kPfRows * kPfCells * 2;   // a P tile (CUDA-core P V only): two boxes
-  static constexpr int NS = 3;                           // K/V stages (one tile each): K, V, V
+  static constexpr int NK = D == 64 ? 3 : 2;             // K ring stages (one tile each)
+  static constexpr int NV = D == 64 ? 4 : 3;             // V ring stages
   static constexpr int OFF_Q = 0;                        // [2 slots][TILE]
-  static constexpr int OFF_P = OFF_Q + 2 * TILE;         // [2 slots][PTILE]
-  static constexpr int OFF_KV = OFF_P + 2 * PTILE;       // [NS][TILE]
-  static constexpr int OFF_BAR = OFF_KV + NS * TILE;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], mma_done
-  static constexpr int N_BAR = 1 + 2 * NS + 6 + 1;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;         // [NK][TILE]
+  static constexpr int OFF_V = OFF_K + NK * TILE;        // [NV][TILE]
+  static constexpr int OFF_BAR = OFF_V + NV * TILE;
+  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
+  // p_full[2], pv_done[2], mma_done, stall (never arrived at: the bounded-wait test)
+  static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 6 + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;   // TMEM base address, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
@@ -224,25 +285,50 @@ __device__ __forceinline__ unsigned char* pf_align1024(unsigned char* p) {
   return p + (((a + 1023u) & ~1023u) - a);
 }
 
-// K/V ring: stage 0 holds the K tile of the current cell tile (one buffer,
-// refilled as soon as every head's S of that tile has completed, so the next K
-// streams in during the softmax); stages 1 and 2 hold V, tile j in stage
-// 1 + (j & 1), refilled once P V two tiles back has completed.  Neither load
-// waits on the tensor core's most recent work.
-__device__ __forceinline__ int pf_vstage(int64_t j) { return 1 + (int)(j & 1); }
-__device__ __forceinline__ uint32_t pf_vparity(int64_t j) { return (uint32_t)((j >> 1) & 1); }
+// K and V rings: the i-th K (or V) tile the CTA loads goes to stage i % NK
+// (i % NV); its "full" barrier completes phase i / NK for it, and the stage's
+// "empty" barrier completes once the tensor core is done with it (K: every
+// head's S of that tile; V: every head's P V), which the load of tile
+// i + NK (i + NV) waits for.  With two K and three V stages the next tiles
+// stream in a step or more ahead of the MMAs that read them.
+template <int N>
+__device__ __forceinline__ int pf_stage(int64_t i) { return (int)(i % N); }
+template <int N>
+__device__ __forceinline__ uint32_t pf_phase(int64_t i) { return (uint32_t)((i / N) & 1); }
 
-// Bounded wait that also gives up as soon as another thread of the CTA has
-// raised the abort flag.
-__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+struct PfBars {
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *pv_done, *mma_done, *stall;
+};
+template <int D>
+__device__ __forceinline__ PfBars pf_bars(unsigned char* sm) {
+  using L = PfLayout<D>;
+  uint64_t* b = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  PfBars r;
+  r.q_full = b;
+  r.k_full = b + 1;
+  r.k_empty = r.k_full + L::NK;
+  r.v_full = r.k_empty + L::NK;
+  r.v_empty = r.v_full + L::NV;
+  r.s_full = r.v_empty + L::NV;
+  r.p_full = r.s_full + 2;
+  r.pv_done = r.s_full + 4;
+  r.mma_done = r.s_full + 6;
+  r.stall = r.s_full + 7;
+  return r;
+}
+
+// Bounded wait (at most p.wait_ns) that also gives up as soon as another
+// thread of the CTA has raised the abort flag.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, const PrefillPlan& p,
+                                        volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((spin & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_status(status, ATTN_ERR_DEVICE_TIMEOUT);
+      if (global_timer_ns() - t0 > p.wait_ns) {
+        record_status(p.status, ATTN_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
         return false;
       }
@@ -251,9 +337,9 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* sta
 }
 
 // Warp-uniform form: every lane waits; the warp goes on only if all did.
-__device__ __forceinline__ bool pf_wait_warp(uint64_t* bar, uint32_t parity, int* status,
+__device__ __forceinline__ bool pf_wait_warp(uint64_t* bar, uint32_t parity, const PrefillPlan& p,
                                              volatile int* abort_flag) {
-  const bool ok = pf_wait(bar, parity, status, abort_flag);
+  const bool ok = pf_wait(bar, parity, p, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -270,24 +356,11 @@ __device__ __forceinline__ void pf_issue_s(uint32_t d_tmem, uint32_t q_base, uin
   }
 }
 
-// O (TMEM, 128 x D f32) (+)= P (128 x 128, K-major) . V (128 cells x D, D
-// contiguous: MN-major).  V's 8-cell groups are 1024 bytes apart (SBO) and its
-// 64-column boxes one box apart (LBO); 16 cells per MMA.
-template <int D>
-__device__ __forceinline__ void pf_issue_pv(uint32_t d_tmem, uint32_t p_base, uint32_t v_base, uint32_t idesc,
-                                            bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < kPfCells / 16; ++kk) {
-    const uint32_t a_off = (uint32_t)(kk >> 2) * PfLayout<D>::BOX + (uint32_t)(kk & 3) * 32u;
-    umma_ss(d_tmem, umma_desc_sw128(p_base + a_off, 16, 1024),
-            umma_desc_sw128(v_base + (uint32_t)kk * 2048u, PfLayout<D>::BOX, 1024), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-
-// The same with P in tensor memory: P (16-bit, two values per 32-bit column,
-// row i in lane i) sits in the first 64 columns of the head's S region; each
-// MMA takes 16 cells = 8 columns of it.
+// O (TMEM, 128 x D f32) (+)= P . V with P in tensor memory: P (16-bit, two
+// values per 32-bit column, row i in lane i) sits in the first 64 columns of
+// the head's S region, and each MMA takes 16 cells = 8 columns of it.  V (128
+// cells x D, D contiguous) is MN-major: its 8-cell groups are 1024 bytes apart
+// (SBO) and its 64-column boxes one box apart (LBO).
 template <int D>
 __device__ __forceinline__ void pf_issue_pv_ts(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_base, uint32_t idesc,
                                                bool accumulate) {
@@ -593,17 +666,67 @@ __device__ __forceinline__ void pf_weights(const float* x, float boff, float bst
   l += s4.x + s4.y;
 }
 
+// P V on the CUDA cores for one thread's row of a tile whose V holds a
+// non-finite value: o[0..D) (+)= sum over the row's visible cells c of
+// P[c] V[c] (P 16-bit, two per word of pk; V in shared memory, 128-byte
+// swizzled 64-column boxes), so that a cell the row cannot see never reaches
+// it through 0 * NaN.  The cell loop is unrolled so that pk stays in registers.
+template <typename KT, int D>
+__device__ __forceinline__ void pf_pv_cuda_cores(const uint32_t* pk, const uint32_t* vis,
+                                                 const unsigned char* Vs, uint32_t tO, bool first,
+                                                 float factor) {
+  using L = PfLayout<D>;
+#pragma unroll 1
+  for (int ch = 0; ch < D / 32; ++ch) {
+    float o[32];
+    uint32_t ou[32];
+    if (!first) {
+      tmem_ld32(tO + ch * 32, ou);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(ou[e]) * factor;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < kPfCells; ++c) {
+      if (!((vis[c >> 5] >> (c & 31)) & 1u)) continue;
+      const uint32_t w = pk[c >> 1];
+      const float pc = pf_widen<KT>((uint16_t)((c & 1) ? (w >> 16) : (w & 0xffffu)));
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const int d = ch * 32 + q8 * 8;
+        const uint32_t voff = (uint32_t)(d >> 6) * L::BOX + (uint32_t)c * 128u +
+                              ((uint32_t)(((d & 63) >> 3) ^ (c & 7)) << 4);
+        float vf[8];
+        unpack_vec<KT>(*reinterpret_cast<const uint4*>(Vs + voff), vf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[q8 * 8 + e] = fmaf(pc, vf[e], o[q8 * 8 + e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e]);
+    tmem_st32(tO + ch * 32, ou);
+  }
+  tmem_wait_st();
+}
+
 template <typename KT, int D>
 __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& tiles, unsigned char* sm,
-                                           uint64_t* bars, volatile int* abort_flag, uint32_t tmem, int rt,
+                                           const PfBars& B, volatile int* abort_flag, uint32_t tmem, int rt,
                                            int h, int slot, int quarter, int lane) {
   const bool out_vec = p.out_vec != 0, mask_vec = p.mask_vec != 0;
   using L = PfLayout<D>;
-  constexpr int NS = L::NS;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* s_full = bars + 1 + 2 * NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = s_full + 4;
+  uint64_t* s_full = B.s_full;
+  uint64_t* p_full = B.p_full;
+  uint64_t* pv_done = B.pv_done;
+  // Bounded-wait test: wait on a barrier nothing arrives at; the wait gives
+  // up after p.wait_ns, records the timeout and raises the abort flag, and
+  // every role of the CTA then winds down.
+  if (p.test_stall) {
+    if (!pf_wait_warp(B.stall, 0u, p, abort_flag)) return;
+  }
   const int row_t = quarter * 32 + lane;
   const int r = rt * kPfRows + row_t;
   const bool rvalid = r < p.R;
@@ -617,7 +740,6 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
   const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
   const uint32_t tS = lane_base + (uint32_t)slot * 128u;
   const uint32_t tO = lane_base + 256u + (uint32_t)slot * D;
-  unsigned char* Ps = sm + L::OFF_P + slot * L::PTILE;
   const float* mrow = (p.f.mask && rvalid) ? p.f.mask + (int64_t)r * p.f.mask_sr : nullptr;
 
   float m = neg_inf(), l = 0.f, mneg2 = 0.f;    // mneg2 = -m * log2(e) (0 while m = -inf)
@@ -626,11 +748,11 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
   float qn2 = 0.f;   // |q_r|^2 of this row and head (softcap range bound)
   for (int kt = tiles.first(); kt >= 0; kt = tiles.next(kt), ++j) {
     const int code = tiles.code(kt);
-    if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
+    if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p, abort_flag)) { ok = false; break; }
     tc_fence_after();
     if (j == 0 && cap && p.kn2) {
       // the Q tile is resident (its load completed before the first S)
-      if (!pf_wait_warp(&bars[0], 0u, p.status, abort_flag)) { ok = false; break; }
+      if (!pf_wait_warp(B.q_full, 0u, p, abort_flag)) { ok = false; break; }
       const unsigned char* Qs = sm + L::OFF_Q + slot * L::TILE;
       float a = 0.f, b = 0.f;
 #pragma unroll
@@ -748,56 +870,11 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     }
 
     if (code == kTileMixedBadV) {
-      // P row in shared memory (K-major 128-byte-swizzled: cells 0-63 in the
-      // first box, 64-127 in the second; 16-byte chunk k of row t at chunk
-      // k ^ (t & 7)) for the CUDA-core P V below.
-#pragma unroll
-      for (int k8 = 0; k8 < kPfCells / 8; ++k8) {
-        const uint4 w = make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
-        const uint32_t off = (uint32_t)(k8 >> 3) * L::BOX + (uint32_t)row_t * 128u +
-                             ((uint32_t)((k8 & 7) ^ (row_t & 7)) << 4);
-        *reinterpret_cast<uint4*>(Ps + off) = w;
-      }
-      // P V on the CUDA cores over this row's visible cells only.
-      const int stV = pf_vstage(j);
-      if (!pf_wait_warp(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
-      const unsigned char* Vs = sm + L::OFF_KV + stV * L::TILE;
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        float o[32];
-        uint32_t ou[32];
-        if (j > 0) {
-          tmem_ld32(tO + ch * 32, ou);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(ou[e]) * factor;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
-        }
-#pragma unroll 2
-        for (int c = 0; c < kPfCells; ++c) {
-          const uint32_t vw = c < 64 ? (c < 32 ? vis[0] : vis[1]) : (c < 96 ? vis[2] : vis[3]);
-          if (!((vw >> (c & 31)) & 1u)) continue;
-          const uint32_t poff = (uint32_t)(c >> 6) * L::BOX + (uint32_t)row_t * 128u +
-                                ((uint32_t)(((c & 63) >> 3) ^ (row_t & 7)) << 4) + (uint32_t)(c & 7) * 2u;
-          const float pc = pf_widen<KT>(*reinterpret_cast<const uint16_t*>(Ps + poff));
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            const int d = ch * 32 + q8 * 8;
-            const uint32_t voff = (uint32_t)(d >> 6) * L::BOX + (uint32_t)c * 128u +
-                                  ((uint32_t)(((d & 63) >> 3) ^ (c & 7)) << 4);
-            float vf[8];
-            unpack_vec<KT>(*reinterpret_cast<const uint4*>(Vs + voff), vf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[q8 * 8 + e] = fmaf(pc, vf[e], o[q8 * 8 + e]);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e]);
-        tmem_st32(tO + ch * 32, ou);
-      }
-      tmem_wait_st();
+      // P V on the CUDA cores over this row's visible cells only (V(j) is
+      // released by the tensor core's commit after this head's p_full).
+      const int stV = pf_stage<L::NV>(j);
+      if (!pf_wait_warp(&B.v_full[stV], pf_phase<L::NV>(j), p, abort_flag)) { ok = false; break; }
+      pf_pv_cuda_cores<KT, D>(pk, vis, sm + L::OFF_V + stV * L::TILE, tO, j == 0, factor);
     } else {
       // P into the first 64 columns of this head's S region (S is read)
       tmem_st32(tS, pk);
@@ -810,7 +887,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
 
   if (!ok) return;
   if (j > 0) {
-    if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p.status, abort_flag)) return;
+    if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p, abort_flag)) return;
     tc_fence_after();
   }
   // Fold with the sink (an extra logit with no value vector) and normalise.
@@ -852,17 +929,10 @@ __global__ void __launch_bounds__(PfLayout<D>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const PrefillPlan p) {
   using L = PfLayout<D>;
-  constexpr int NS = L::NS;
+  constexpr int NK = L::NK, NV = L::NV;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = pf_align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + NS;
-  uint64_t* s_full = bars + 1 + 2 * NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = s_full + 4;
-  uint64_t* mma_done = s_full + 6;
+  const PfBars B = pf_bars<D>(sm);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
 
@@ -876,14 +946,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int n_slots = two ? 2 : 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < NS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    mbar_init(B.q_full, 1);
+    for (int s = 0; s < NK; ++s) { mbar_init(&B.k_full[s], 1); mbar_init(&B.k_empty[s], 1); }
+    for (int s = 0; s < NV; ++s) { mbar_init(&B.v_full[s], 1); mbar_init(&B.v_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], kPfRows);
-      mbar_init(&pv_done[s], 1);
+      mbar_init(&B.s_full[s], 1);
+      mbar_init(&B.p_full[s], kPfRows);
+      mbar_init(&B.pv_done[s], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(B.mma_done, 1);
+    mbar_init(B.stall, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -901,7 +973,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     setmaxnreg_inc<L::HIGH_REGS>();
     const int slot = (warp >> 2) - 1;
     if (slot < n_slots)
-      pf_softmax<KT, D>(p, tiles, sm, bars, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane);
+      pf_softmax<KT, D>(p, tiles, sm, B, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane);
   } else {
   setmaxnreg_dec<L::LOW_REGS>();
   if (warp == 0) {
@@ -909,39 +981,44 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
       int kt = tiles.first();
-      int64_t nK = 0, nV = 0;   // K and V tile loads issued
+      // K and V loads issued; the i-th goes to K stage i % NK, V stage i % NV
+      int64_t nK = 0, nV = 0;
       const bool any = kt >= 0;
       if (any) {
-        mbar_arrive_expect_tx(q_full, (uint32_t)(n_slots * L::TILE));
+        mbar_arrive_expect_tx(B.q_full, (uint32_t)(n_slots * L::TILE));
         for (int s = 0; s < n_slots; ++s)
 #pragma unroll
           for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, q_full, bx * 64, h0 + s, rt * kPfRows,
+            tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, B.q_full, bx * 64, h0 + s, rt * kPfRows,
                         pol);
       }
       for (; kt >= 0; kt = tiles.next(kt)) {
-        // K of this tile once every head's S of the previous tile is done
-        if (nK >= 1 && !pf_wait(&kv_empty[0], (uint32_t)((nK - 1) & 1), p.status, abort_flag)) break;
-        mbar_arrive_expect_tx(&kv_full[0], (uint32_t)L::TILE);
+        // K of this tile once every head's S of the tile NK loads back is done
+        const int sk = pf_stage<NK>(nK);
+        if (nK >= NK && !pf_wait(&B.k_empty[sk], pf_phase<NK>(nK - NK), p, abort_flag)) break;
+        mbar_arrive_expect_tx(&B.k_full[sk], (uint32_t)L::TILE);
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_3d(sm + L::OFF_KV + bx * L::BOX, &tmK, &kv_full[0], bx * 64, g, kt * kPfCells, pol);
+          tma_load_3d(sm + L::OFF_K + sk * L::TILE + bx * L::BOX, &tmK, &B.k_full[sk], bx * 64, g, kt * kPfCells,
+                      pol);
         ++nK;
-        // V of this tile once P V two tiles back is done
-        const int sv = pf_vstage(nV);
-        if (nV >= 2 && !pf_wait(&kv_empty[sv], (uint32_t)(((nV >> 1) - 1) & 1), p.status, abort_flag)) break;
-        mbar_arrive_expect_tx(&kv_full[sv], (uint32_t)L::TILE);
+        // V of this tile once every head's P V of the tile NV loads back is done
+        const int sv = pf_stage<NV>(nV);
+        if (nV >= NV && !pf_wait(&B.v_empty[sv], pf_phase<NV>(nV - NV), p, abort_flag)) break;
+        mbar_arrive_expect_tx(&B.v_full[sv], (uint32_t)L::TILE);
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_3d(sm + L::OFF_KV + sv * L::TILE + bx * L::BOX, &tmV, &kv_full[sv], bx * 64, g, kt * kPfCells,
+          tma_load_3d(sm + L::OFF_V + sv * L::TILE + bx * L::BOX, &tmV, &B.v_full[sv], bx * 64, g, kt * kPfCells,
                       pol);
         ++nV;
       }
-      // leave no copy in flight (bounded; completed loads return at once)
-      if (nK >= 1) mbar_wait_bounded(&kv_full[0], (uint32_t)((nK - 1) & 1), nullptr);
-      for (int64_t k = nV > 2 ? nV - 2 : 0; k < nV; ++k)
-        mbar_wait_bounded(&kv_full[pf_vstage(k)], pf_vparity(k), nullptr);
-      if (any) mbar_wait_bounded(q_full, 0, nullptr);
+      // Leave no copy in flight (bounded; completed loads return at once):
+      // the last NK K loads and the last NV V loads issued.
+      for (int64_t k = nK > NK ? nK - NK : 0; k < nK; ++k)
+        mbar_wait_bounded(&B.k_full[pf_stage<NK>(k)], pf_phase<NK>(k), nullptr);
+      for (int64_t k = nV > NV ? nV - NV : 0; k < nV; ++k)
+        mbar_wait_bounded(&B.v_full[pf_stage<NV>(k)], pf_phase<NV>(k), nullptr);
+      if (any) mbar_wait_bounded(B.q_full, 0, nullptr);
     }
   } else if (warp == 1) {
     // ---- MMA issuer ----
@@ -950,48 +1027,49 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t idS = umma_idesc_f16(kPfRows, kPfCells, bf, 0, 0);
       constexpr uint32_t idO = umma_idesc_f16(kPfRows, D, bf, 0, 1);
       const uint32_t q_addr = smem_u32(sm + L::OFF_Q);
-      const uint32_t kv_addr = smem_u32(sm + L::OFF_KV);
+      const uint32_t k_addr = smem_u32(sm + L::OFF_K);
+      const uint32_t v_addr = smem_u32(sm + L::OFF_V);
       int kt = tiles.first();
       bool ok = kt >= 0;
       if (ok) {
-        ok = pf_wait(q_full, 0, p.status, abort_flag) && pf_wait(&kv_full[0], 0, p.status, abort_flag);
+        ok = pf_wait(B.q_full, 0, p, abort_flag) && pf_wait(&B.k_full[0], 0, p, abort_flag);
         if (ok) {
           tc_fence_after();
           for (int s = 0; s < n_slots; ++s) {
-            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr, idS);
-            umma_commit(&s_full[s]);
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, k_addr, idS);
+            umma_commit(&B.s_full[s]);
           }
-          umma_commit(&kv_empty[0]);
+          umma_commit(&B.k_empty[0]);
         }
       }
       for (int64_t j = 0; ok && kt >= 0; ++j) {
         const int kn = tiles.next(kt);
         const bool has_next = kn >= 0;
         const bool pv_mma = tiles.code(kt) != kTileMixedBadV;
-        const int stV = pf_vstage(j);
+        const int stV = pf_stage<NV>(j), stK = pf_stage<NK>(j + 1);
         // per head: P V of this tile (P in the head's S columns), then the
         // next tile's S over them
         for (int s = 0; s < n_slots && ok; ++s) {
-          if (!pf_wait(&p_full[s], (uint32_t)(j & 1), p.status, abort_flag)) { ok = false; break; }
-          if (s == 0 && !pf_wait(&kv_full[stV], pf_vparity(j), p.status, abort_flag)) { ok = false; break; }
+          if (!pf_wait(&B.p_full[s], (uint32_t)(j & 1), p, abort_flag)) { ok = false; break; }
+          if (s == 0 && !pf_wait(&B.v_full[stV], pf_phase<NV>(j), p, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if (pv_mma)
-            pf_issue_pv_ts<D>(tmem + 256u + (uint32_t)s * D, tmem + (uint32_t)s * 128u, kv_addr + stV * L::TILE,
+            pf_issue_pv_ts<D>(tmem + 256u + (uint32_t)s * D, tmem + (uint32_t)s * 128u, v_addr + stV * L::TILE,
                               idO, j > 0);
-          umma_commit(&pv_done[s]);
+          umma_commit(&B.pv_done[s]);
           if (has_next) {
-            if (s == 0 && !pf_wait(&kv_full[0], (uint32_t)((j + 1) & 1), p.status, abort_flag)) { ok = false; break; }
+            if (s == 0 && !pf_wait(&B.k_full[stK], pf_phase<NK>(j + 1), p, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, kv_addr, idS);
-            umma_commit(&s_full[s]);
-            if (s == n_slots - 1) umma_commit(&kv_empty[0]);
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, k_addr + stK * L::TILE, idS);
+            umma_commit(&B.s_full[s]);
+            if (s == n_slots - 1) umma_commit(&B.k_empty[stK]);
           }
         }
         if (!ok) break;
-        umma_commit(&kv_empty[stV]);
+        umma_commit(&B.v_empty[stV]);
         kt = kn;
       }
-      umma_commit(mma_done);   // arrives once every MMA issued above has retired
+      umma_commit(B.mma_done);   // arrives once every MMA issued above has retired
     }
   }   // warps 2 and 3 have no role
   }
@@ -1000,7 +1078,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    mbar_wait_bounded(mma_done, 0, p.status);
+    mbar_wait_bounded(B.mma_done, 0, p.status);
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
@@ -1015,7 +1093,7 @@ cudaError_t launch_prefill_t(const PrefillPlan& p, const CUtensorMap& tmQ, const
   if (e != cudaSuccess) return e;
   const int64_t n_cls = (int64_t)p.n_rt * p.n_kt, n_scan = (int64_t)p.n_kt * p.Hkv;
   if (n_cls + n_scan > 0) {
-    prefill_classify_kernel<<<(unsigned)(n_cls + n_scan), 256, 0, stream>>>(p);
+    prefill_classify_kernel<<<(unsigned)(n_cls + n_scan), kClsThreads, 0, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (after_classify) cudaEventRecord(after_classify, stream);

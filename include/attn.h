@@ -156,7 +156,15 @@ typedef struct {
     int32_t grid_order;   /* 0: rows vary fastest over the (rows, heads, slices)
                              grid; 1: slices fastest.  Results are bit-identical;
                              exposed for tests and tuning.                           */
-    int32_t reserved[5];  /* must be zero                                            */
+    int32_t reserved[5];  /* must be zero, except reserved[0] in attn_prefill: a
+                             test of the kernels' bounded waits.  A value t in
+                             1..1000000 makes every CTA of the dense tensor-core
+                             prefill first wait, for at most t microseconds, on
+                             a barrier nothing arrives at; the wait gives up,
+                             the CTA winds down (no copy left in flight, tensor
+                             memory freed) without writing its output, and
+                             attn_check_device_status() then reports
+                             ATTN_ERR_DEVICE_TIMEOUT.  For tests only.      */
 
     const float *k_scale, *v_scale;   /* quantized caches: per (cell, KV head) scales, else NULL */
     int64_t scale_stride_cell;        /* elements between cells' scale rows (>= n_head_kv)   */

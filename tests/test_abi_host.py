@@ -115,6 +115,22 @@ def test_validation_pairs_and_reserved(lib):
     assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1
 
 
+def test_bounded_wait_test_field(lib):
+    """reserved[0] is the prefill kernel's bounded-wait test (microseconds,
+    0..1000000); every other op and field still takes zero only."""
+    a = _args(q_type=A.ATTN_BF16, kv_type=A.ATTN_BF16)
+    a.reserved[0] = 1000
+    assert lib.attn_supports(ctypes.byref(a), A.OP_PREFILL) == 0
+    assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1
+    assert lib.attn_supports(ctypes.byref(a), A.OP_SELECTED) == -1
+    for bad in (-1, 1000001):
+        a.reserved[0] = bad
+        assert lib.attn_supports(ctypes.byref(a), A.OP_PREFILL) == -1
+    a.reserved[0] = 1000
+    a.cell_seq, a.row_seq = 0x50000, 0x60000      # the unified-cache route has no such wait
+    assert lib.attn_supports(ctypes.byref(a), A.OP_PREFILL) == -1
+
+
 def test_quantized_cache_validation(lib):
     """e4m3/int8 caches: decode only, scales required, and only for such caches."""
     for kv in (A.ATTN_FP8_E4M3, A.ATTN_I8):
