@@ -236,7 +236,11 @@ DecodeShape plan_decode(const attn_args* a, int sms) {
   DecodeShape d;
   const int G = a->n_head_q / a->n_head_kv;
   d.mma = decode_uses_mma(a->kv_type, a->q_type, a->q, a->q_stride_row, a->q_stride_head);
-  d.stream = d.mma && a->n_slices == 0;
+  // one-byte caches take the balanced tensor-core kernel too (codes widened
+  // to f16 in registers); forced slice counts keep the CUDA-core grid kernel
+  const bool mma8 = a->n_slices == 0 && decode_stream8_supported(a->kv_type, a->q_type, a->q, a->q_stride_row,
+                                                                 a->q_stride_head, a->head_dim, G);
+  d.stream = (d.mma && a->n_slices == 0) || mma8;
   d.hg = G > 8 ? 2 : 1;
   d.hpw = G > 8 ? 8 : pick_hpw(G);
   d.W = d.stream ? decode_stream_warps(a->kv_type, a->head_dim, G, sms) : 0;
@@ -366,8 +370,8 @@ int32_t check_prefill(const attn_args* a) {
   if (a->kv_type != ATTN_F16 && a->kv_type != ATTN_BF16)
     return fail(ATTN_ERR_UNSUPPORTED, "prefill: K/V must be F16 or BF16");
   if (a->q_type != a->kv_type) return fail(ATTN_ERR_UNSUPPORTED, "prefill: Q must be in the K/V dtype");
-  if (a->head_dim != 64 && a->head_dim != 128)
-    return fail(ATTN_ERR_UNSUPPORTED, "prefill: head_dim %d not in {64, 128}", a->head_dim);
+  if (a->head_dim != 64 && a->head_dim != 128 && a->head_dim != 256)
+    return fail(ATTN_ERR_UNSUPPORTED, "prefill: head_dim %d not in {64, 128, 256}", a->head_dim);
   if (a->reserved[0] < 0 || a->reserved[0] > 1000000)
     return fail(ATTN_ERR_INVALID_ARG, "prefill: reserved[0] (the bounded-wait test) must be 0..1000000 us");
   if (a->reserved[0] != 0 && unified_route(a))
@@ -380,7 +384,7 @@ int32_t check_prefill(const attn_args* a) {
   }
   const int64_t n_rt = ((int64_t)a->n_rows + kPfTile - 1) / kPfTile;
   const int G = a->n_head_q / a->n_head_kv;
-  const int64_t ctas = n_rt * a->n_head_kv * ((G + 1) / 2);
+  const int64_t ctas = n_rt * a->n_head_kv * (a->head_dim <= 128 ? (G + 1) / 2 : G);
   const int64_t n_kt = ((int64_t)a->n_cells + kPfTile - 1) / kPfTile;
   if (ctas > 0x7fffffffLL || n_rt * n_kt + n_kt * a->n_head_kv > 0x7fffffffLL)
     return fail(ATTN_ERR_UNSUPPORTED, "prefill: grid too large");
@@ -571,16 +575,20 @@ int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* s
   if (blocks > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid of %lld CTAs is too large", (long long)blocks);
 
   const bool mma = sh.mma;
+  // tile maps: tensor-core kernels take 16-cell tiles in 128-byte swizzled
+  // boxes (64 16-bit values or 128 one-byte codes per cell); the CUDA-core
+  // grid kernel takes 32-cell tiles of whole rows
+  const bool tc = sh.stream || mma;
   CUtensorMap tmK, tmV;
   memset(&tmK, 0, sizeof(tmK));
   memset(&tmV, 0, sizeof(tmV));
   if (a->n_cells > 0) {
-    const int box_d = mma ? 64 : 0;
+    const int box_d = !tc ? 0 : dtype_size(a->kv_type) == 1 ? 128 : 64;
     if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
-                          a->kv_stride_head, mma ? 16 : 32, box_d, mma)) != ATTN_OK)
+                          a->kv_stride_head, tc ? 16 : 32, box_d, tc)) != ATTN_OK)
       return st;
     if ((st = make_kv_map(&tmV, a->v, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
-                          a->kv_stride_head, mma ? 16 : 32, box_d, mma)) != ATTN_OK)
+                          a->kv_stride_head, tc ? 16 : 32, box_d, tc)) != ATTN_OK)
       return st;
   }
 
@@ -747,7 +755,7 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
   p.n_rt = (a->n_rows + kPfTile - 1) / kPfTile;
   p.n_kt = (a->n_cells + kPfTile - 1) / kPfTile;
-  p.n_pairs = (p.G + 1) / 2;
+  p.n_pairs = a->head_dim <= 128 ? (p.G + 1) / 2 : p.G;   // q heads per CTA: 2 up to head dim 128, 1 at 256
   char* wsb = static_cast<char*>(ws);
   p.cls = reinterpret_cast<uint8_t*>(wsb);
   p.vbad = reinterpret_cast<uint8_t*>(wsb + wl.vbad_off);
@@ -778,9 +786,28 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
       p.s_lim = (float)s_lim;
       p.bound2 = (float)(0.998 * s_lim * s_lim);
       p.cap_raw = 1;
+      // bound path: the same series with log2(e) folded in; degree 7 for
+      // |u| <= c / 3 (the next term, 62/2835 (1/3)^9 c, is below 1e-6 c)
+      const double L = 1.4426950408889634, s7 = c / (3.0 * std::fabs(sc));
+      p.b3 = (float)(a3 * L);
+      p.b5 = (float)(a5 * L);
+      p.b7 = (float)(a7 * L);
+      p.b9 = (float)(a9 * L);
+      p.bound7 = normal(s7 * s7) ? (float)(0.998 * s7 * s7) : -1.f;
     }
   }
-  if (!p.cap_raw) p.kn2 = nullptr;   // the tile norms serve the packed softcap only
+  // Bound path of bf16 prefill: logits bounded through |q| max|k| (needs a
+  // finite scale); the packed softcap also uses the tile norms.
+  const bool scale_ok = std::isfinite(a->scale);
+  p.bsc = (float)((double)a->scale * 1.4426950408889634);
+  // |scale| |q| max|k| <= 30: the bound then sits within 60 of the tile's
+  // true max, so no visible weight underflows
+  const double s2 = (double)a->scale * a->scale;
+  const double lim2 = s2 > 0.0 ? 900.0 / s2 : 1e30;
+  p.nc_lim2 = scale_ok ? (float)std::min(lim2, 1e30) : -1.f;
+  p.bound7 = scale_ok ? std::min(p.bound7, p.nc_lim2) : -1.f;
+  p.bound9 = scale_ok && p.cap_raw ? std::min(p.bound2, p.nc_lim2) : -1.f;
+  if (!p.cap_raw && a->kv_type != ATTN_BF16) p.kn2 = nullptr;
   const int oes = dtype_size(a->out_type);
   const int64_t ovec = 16 / oes;
   p.out_vec = aligned16(a->out) && (a->n_rows <= 1 || a->o_stride_row % ovec == 0) &&

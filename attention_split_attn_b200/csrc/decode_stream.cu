@@ -1,5 +1,7 @@
 // decode_stream.cu -- balanced persistent split-K decode for 16-bit caches
-// (attn_decode with n_slices == 0 and Q in the cache dtype).
+// (attn_decode with n_slices == 0 and Q in the cache dtype) and for one-byte
+// caches (e4m3 / int8 codes with per (cell, KV head) scales, Q in bf16 or
+// f16; the tile step of decode_tile8.cuh).
 //
 // The split-K idea of the pages (TensorFold PR #2595: split each row's keys
 // into slices, fold the slice partials afterwards) with slices sized for the
@@ -25,8 +27,10 @@
 // computes the prefix itself and no planner runs.
 #include "common.cuh"
 #include "decode_tile.cuh"
+#include "decode_tile8.cuh"
 #include "internal.h"
 #include "mma.cuh"
+#include "quant.cuh"
 
 namespace attn {
 
@@ -36,13 +40,49 @@ namespace {
 // planner kernel in front of the stream kernel).
 constexpr int kInlineRows = 64;
 
-template <int D>
+// The tile step of a cache type: decode_tile.cuh for 16-bit values,
+// decode_tile8.cuh for one-byte codes; ES bytes per element, so a stage is
+// 16 cells x D elements of K then of V, each in D ES / 128 TMA boxes of 128
+// bytes per cell.
+template <typename KT, int D, int NH>
+struct StreamTraits {
+  using State = WarpTileState<KT, D, NH>;
+  static constexpr int ES = 2;
+};
+template <int D, int NH>
+struct StreamTraits<e4m3_code, D, NH> {
+  using State = WarpTileState8<e4m3_code, D, NH>;
+  static constexpr int ES = 1;
+};
+template <int D, int NH>
+struct StreamTraits<i8_code, D, NH> {
+  using State = WarpTileState8<i8_code, D, NH>;
+  static constexpr int ES = 1;
+};
+
+template <int D, int ES>
 struct StreamRing {
   static constexpr int NS = 2;                       // ring stages per warp
-  static constexpr int BAR_OFF = NS * WarpStage<D>::BYTES;
+  static constexpr int TILE = kWarpTile * D * ES;    // K (or V) of one tile
+  static constexpr int STAGE = 2 * TILE;
+  static constexpr int BAR_OFF = NS * STAGE;
   static constexpr int RT_OFF = BAR_OFF + NS * 8;    // inline row tile prefix [kInlineRows + 1]
   static constexpr int TOTAL = RT_OFF + (kInlineRows + 1) * 8 + 1024;   // + alignment slack for the swizzle
 };
+
+// TMA of one 16-cell K/V tile of KV head g starting at cell c0 (boxes of 128
+// bytes per cell, 128-byte swizzled, each sub-tile 16 x 128 B).
+template <int D, int ES>
+__device__ __forceinline__ void issue_stream_tile(unsigned char* stage, uint64_t* bar, const CUtensorMap* tmK,
+                                                  const CUtensorMap* tmV, int g, int c0, uint64_t pol) {
+  constexpr int TILE = kWarpTile * D * ES, NB = D * ES / 128, EPB = 128 / ES;
+  mbar_arrive_expect_tx(bar, 2 * TILE);
+#pragma unroll
+  for (int sub = 0; sub < NB; ++sub) {
+    tma_load_3d(stage + sub * (kWarpTile * 128), tmK, bar, sub * EPB, g, c0, pol);
+    tma_load_3d(stage + TILE + sub * (kWarpTile * 128), tmV, bar, sub * EPB, g, c0, pol);
+  }
+}
 
 __device__ __forceinline__ int64_t row_len(const DecodePlan& p, int r) {
   int32_t b = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
@@ -123,10 +163,12 @@ template <typename KT, int D, int NH>
 __global__ void __launch_bounds__(32)
 decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodePlan p) {
-  constexpr int NS = StreamRing<D>::NS;
+  using Tr = StreamTraits<KT, D, NH>;
+  using Ring = StreamRing<D, Tr::ES>;
+  constexpr int NS = Ring::NS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + StreamRing<D>::BAR_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ring::BAR_OFF);
   const int lane = threadIdx.x;
   if (lane == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
@@ -139,7 +181,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   // reading a workspace this call is about to reuse.
   const int64_t* row_tiles = p.row_tiles;
   if (p.plan_inline) {
-    int64_t* rt = reinterpret_cast<int64_t*>(smem + StreamRing<D>::RT_OFF);
+    int64_t* rt = reinterpret_cast<int64_t*>(smem + Ring::RT_OFF);
     int64_t carry = 0;
     for (int base = 0; base < p.R; base += 32) {
       const int r = base + lane;
@@ -200,8 +242,8 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     pol = policy_evict_first();
     for (; issued < (n < NS ? n : (int64_t)NS); ++issued) {
       if (issued > 0) cursor_next(p, row_tiles, ic);
-      issue_warp_tile<D>(smem + issued * WarpStage<D>::BYTES, &full[issued], &tmK, &tmV, ic.g,
-                         ic.begin + (int)(ic.j * kWarpTile), pol);
+      issue_stream_tile<D, Tr::ES>(smem + issued * Ring::STAGE, &full[issued], &tmK, &tmV, ic.g,
+                                   ic.begin + (int)(ic.j * kWarpTile), pol);
     }
   }
 
@@ -218,7 +260,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     return rc;
   };
   RowCtx rc = make_ctx(c);
-  WarpTileState<KT, D, NH> st;
+  typename Tr::State st;
   st.reset();
   st.init_offsets(lane);
   st.load_q(p, c.r, c.g * p.G, lane);
@@ -231,7 +273,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       aborted = true;
       break;
     }
-    unsigned char* stage = smem + stg * WarpStage<D>::BYTES;
+    unsigned char* stage = smem + stg * Ring::STAGE;
     st.load_tile(stage);
     auto refill = [&]() {
       __syncwarp();
@@ -239,7 +281,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         // the lanes' shared-memory reads of this stage precede its async refill
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         cursor_next(p, row_tiles, ic);
-        issue_warp_tile<D>(stage, &full[stg], &tmK, &tmV, ic.g, ic.begin + (int)(ic.j * kWarpTile), pol);
+        issue_stream_tile<D, Tr::ES>(stage, &full[stg], &tmK, &tmV, ic.g, ic.begin + (int)(ic.j * kWarpTile), pol);
         ++issued;
       }
     };
@@ -279,8 +321,9 @@ template <typename KT, int D, int NH>
 cudaError_t launch_stream_t(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             cudaStream_t stream, cudaEvent_t after_main) {
   auto kern = decode_stream_kernel<KT, D, NH>;
+  using Ring = StreamRing<D, StreamTraits<KT, D, NH>::ES>;
   static std::atomic<unsigned long long> smem_set{0ull};
-  cudaError_t e = set_smem_limit_once(smem_set, kern, StreamRing<D>::TOTAL);
+  cudaError_t e = set_smem_limit_once(smem_set, kern, Ring::TOTAL);
   if (e != cudaSuccess) return e;
   if (!p.plan_inline) {
     decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
@@ -289,7 +332,7 @@ cudaError_t launch_stream_t(const DecodePlan& p, const CUtensorMap& tmK, const C
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.W);
   cfg.blockDim = dim3(32);
-  cfg.dynamicSmemBytes = StreamRing<D>::TOTAL;
+  cfg.dynamicSmemBytes = Ring::TOTAL;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -319,10 +362,13 @@ cudaError_t launch_stream_k(const DecodePlan& p, const CUtensorMap& tmK, const C
 template <typename KT, int D, int NH>
 int stream_blocks_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<KT, D, NH>, 32,
-                                                    StreamRing<D>::TOTAL) != cudaSuccess || n <= 0) {
+  using Ring = StreamRing<D, StreamTraits<KT, D, NH>::ES>;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_kernel<KT, D, NH>, 32, Ring::TOTAL) !=
+          cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
     // no device: the shared-memory bound of a 228 KB SM with 1 KB reserved per CTA
-    n = (228 * 1024) / (StreamRing<D>::TOTAL + 1024);
+    n = (228 * 1024) / (Ring::TOTAL + 1024);
   }
   return n;
 }
@@ -332,7 +378,11 @@ int stream_blocks_per_sm() {
 int decode_stream_warps(int kv_type, int D, int G, int sms) {
   int per_sm;
   const bool h16 = G > 8;
-  if (kv_type == ATTN_F16) {
+  if (kv_type == ATTN_FP8_E4M3 || kv_type == ATTN_I8) {
+    const bool e4 = kv_type == ATTN_FP8_E4M3;
+    per_sm = D == 128 ? (e4 ? stream_blocks_per_sm<e4m3_code, 128, 8>() : stream_blocks_per_sm<i8_code, 128, 8>())
+                      : (e4 ? stream_blocks_per_sm<e4m3_code, 256, 8>() : stream_blocks_per_sm<i8_code, 256, 8>());
+  } else if (kv_type == ATTN_F16) {
     per_sm = D == 64 ? (h16 ? stream_blocks_per_sm<__half, 64, 16>() : stream_blocks_per_sm<__half, 64, 8>())
            : D == 128 ? (h16 ? stream_blocks_per_sm<__half, 128, 16>() : stream_blocks_per_sm<__half, 128, 8>())
                       : (h16 ? stream_blocks_per_sm<__half, 256, 16>() : stream_blocks_per_sm<__half, 256, 8>());
@@ -344,8 +394,24 @@ int decode_stream_warps(int kv_type, int D, int G, int sms) {
   return std::max(1, per_sm) * std::max(1, sms);
 }
 
+bool decode_stream8_supported(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh, int D, int G) {
+  // one-byte caches on the tensor cores: head dim 128 or 256, up to 8 q heads
+  // per KV head, Q in bf16 or f16 with 16-byte-aligned rows
+  return (kv_type == ATTN_FP8_E4M3 || kv_type == ATTN_I8) && (q_type == ATTN_BF16 || q_type == ATTN_F16) &&
+         (D == 128 || D == 256) && G >= 1 && G <= 8 && (reinterpret_cast<uintptr_t>(q) & 15u) == 0 &&
+         q_sr % 8 == 0 && q_sh % 8 == 0;
+}
+
 cudaError_t launch_decode_stream(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                  cudaStream_t stream, cudaEvent_t after_main) {
+  if (p.kv_type == ATTN_FP8_E4M3 || p.kv_type == ATTN_I8) {
+    const bool e4 = p.kv_type == ATTN_FP8_E4M3;
+    if (p.D == 128)
+      return e4 ? launch_stream_t<e4m3_code, 128, 8>(p, tmK, tmV, stream, after_main)
+                : launch_stream_t<i8_code, 128, 8>(p, tmK, tmV, stream, after_main);
+    return e4 ? launch_stream_t<e4m3_code, 256, 8>(p, tmK, tmV, stream, after_main)
+              : launch_stream_t<i8_code, 256, 8>(p, tmK, tmV, stream, after_main);
+  }
   if (p.kv_type == ATTN_F16) return launch_stream_k<__half>(p, tmK, tmV, stream, after_main);
   return launch_stream_k<__nv_bfloat16>(p, tmK, tmV, stream, after_main);
 }

@@ -80,6 +80,8 @@ cudaError_t launch_decode_slices(const DecodePlan& p, const CUtensorMap& tmK, co
 // Balanced persistent scheme: planner kernel, then W single-warp CTAs that
 // each take an equal run of the flattened (row, KV head, 16-cell tile) space.
 int decode_stream_warps(int kv_type, int D, int G, int sms);
+// One-byte caches (e4m3 / int8) that the balanced tensor-core kernel takes.
+bool decode_stream8_supported(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh, int D, int G);
 cudaError_t launch_decode_stream(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                  cudaStream_t stream, cudaEvent_t after_main);
 
@@ -143,7 +145,7 @@ struct PrefillPlan {
   RowFilter f;
   Logits lg;
   int32_t n_rt, n_kt;       // row tiles, cell tiles (128 each)
-  int32_t n_pairs;          // ceil(G / 2): CTAs per (row tile, KV head)
+  int32_t n_pairs;          // CTAs per (row tile, KV head): ceil(G / 2) up to head dim 128, G at 256
   uint8_t* cls;             // workspace [n_rt][n_kt]
   uint32_t* bits;           // workspace [n_rt][n_kt][128 rows][4 words] (with a mask) or NULL
   uint8_t* vbad;            // workspace [n_kt][Hkv]
@@ -160,6 +162,11 @@ struct PrefillPlan {
   // for every row: |q_r|^2 max_c |k_c|^2 <= bound2 (= 0.998 s_lim^2).
   float bound2;
   float* kn2;               // workspace [n_kt][Hkv]: max |k_c|^2 over the tile (NaN/inf kept)
+  // Bound path (bf16 K/V): the softcap constants times log2(e) (b_n = a_n log2 e,
+  // bsc = scale log2 e) and the |q|^2 max|k|^2 limits under which it runs:
+  // degree-7 series (bound7: |u| <= c / 3), degree 9 (bound9: |u| <= 0.4 c),
+  // no softcap (nc_lim2); each also keeps |scale| |q| max|k| <= 30.
+  float b3, b5, b7, b9, bsc, bound7, bound9, nc_lim2;
   int32_t out_vec;          // output rows may be written with 16-byte stores
   int32_t mask_vec;         // mask rows may be read with 16-byte loads
   int* status;

@@ -58,6 +58,11 @@ namespace {
 constexpr int kPfRows = 128;   // query rows per tile (MMA M)
 constexpr int kPfCells = 128;  // cells per tile (MMA N of S, K of P V)
 
+__device__ __forceinline__ unsigned char* pf_align1024(unsigned char* p) {
+  const uint32_t a = smem_u32(p);
+  return p + (((a + 1023u) & ~1023u) - a);
+}
+
 // ---------------------------------------------------------------------------
 // tile classifier
 // ---------------------------------------------------------------------------
@@ -75,27 +80,17 @@ __device__ __forceinline__ RowVis row_vis(const RowFilter& f, int r, int N) {
   return v;
 }
 
-// Blocks (rt, kt) for blockIdx.x < n_rt * n_kt classify one tile each; blocks
-// (kt, g) after them scan one cell tile of one KV head.  256 threads.
-//  * Classification: the 128 rows' range, sequence and position are staged in
-//    shared memory; warp w takes rows w, w + 8, ..., lane l cells 4l .. 4l + 3
-//    of the tile, and with a mask each warp issues its 16 rows' 16-byte mask
-//    loads before using any of them (the scan is bound by DRAM latency
-//    otherwise).  A row's visibility bits are gathered from the lanes' nibbles
-//    by three shuffles per 8-lane group (word k = cells 32k .. 32k + 31).
-//  * V scan and K norms: every 16-byte chunk of the tile's V and K rows of
-//    head g is loaded before any is used.
+// Classification of tile b = (rt, kt) by one CTA of 256 threads: the 128
+// rows' range, sequence and position are staged in shared memory; warp w
+// takes rows w, w + 8, ..., lane l cells 4l .. 4l + 3 of the tile, and each
+// warp issues its 16 rows' 16-byte mask loads before using any of them (the
+// scan is bound by DRAM latency otherwise).  A row's visibility bits are gathered from the lanes'
+// nibbles by three shuffles per 8-lane group (word k = cells 32k .. 32k + 31).
 constexpr int kClsThreads = 256;
 constexpr int kClsRowsPerWarp = kPfRows / (kClsThreads / 32);   // 16
 
-__global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPlan p) {
-  pdl_launch_dependents();   // the prefill kernel may start its prologue
-  __shared__ int4 rows_sh[kPfRows];
-  __shared__ float wmax[kClsThreads / 32];
+__device__ __forceinline__ void pf_classify_tile(const PrefillPlan& p, int64_t b, int4* rows_sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t b = blockIdx.x;
-  const int64_t n_cls = (int64_t)p.n_rt * p.n_kt;
-  if (b < n_cls) {
     const int rt = (int)(b / p.n_kt), kt = (int)(b % p.n_kt);
     if (tid < kPfRows) {
       const int r = rt * kPfRows + tid;
@@ -175,64 +170,71 @@ __global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPl
       const int cl = !a ? kTileSkip : !nf ? kTileFull : (p.bits && !bs) ? kTileBits : kTileMixed;
       p.cls[b] = (uint8_t)(cl | (lt ? kTileLate : 0));
     }
-  } else {
-    const int64_t vb = b - n_cls;
-    const int kt = (int)(vb / p.Hkv), g = (int)(vb % p.Hkv);
+}
+
+// V scan and K norms of cell tile kt for KV head g by one CTA: every 16-byte
+// chunk of a round is loaded before any is used.
+__device__ __forceinline__ void pf_scan_tile(const PrefillPlan& p, int kt, int g, float* wmax) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // 16-byte chunks of the tile's rows of head g: 128 cells x D/8 chunks,
     // chunk i of this thread = tid + 256 i (per_row chunks of one cell sit in
     // per_row consecutive lanes; per_row divides 32).
     const int per_row = p.D / 8;
     const int n_chunk = kPfCells * per_row;
-    constexpr int kMaxPer = kPfCells * 16 / kClsThreads;   // D <= 128
+    constexpr int kPer = 8;   // chunks per thread per round (all loads of a round go out first)
     const uint16_t* vbase = static_cast<const uint16_t*>(p.v) + (int64_t)g * p.kv_sh;
     const uint16_t* kbase = static_cast<const uint16_t*>(p.k) + (int64_t)g * p.kv_sh;
-    uint4 vw[kMaxPer], kw[kMaxPer];
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) {
-      const int i = tid + k * kClsThreads;
-      const int c = kt * kPfCells + i / per_row;
-      vw[k] = make_uint4(0u, 0u, 0u, 0u);
-      kw[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (i < n_chunk && c < p.N) {
-        vw[k] = __ldg(reinterpret_cast<const uint4*>(vbase + (int64_t)c * p.kv_sc) + (i % per_row));
-        if (p.kn2) kw[k] = __ldg(reinterpret_cast<const uint4*>(kbase + (int64_t)c * p.kv_sc) + (i % per_row));
-      }
-    }
     // A 16-bit value is non-finite iff its exponent field is all ones.
     const uint32_t e_lo = p.kv_type == ATTN_BF16 ? 0x7F80u : 0x7C00u;
     bool bad = false;
+    float mx = 0.f;   // max over the tile's cells of |k_c|^2 (NaN-propagating)
+    for (int base = 0; base < n_chunk; base += kPer * kClsThreads) {
+      uint4 vw[kPer], kw[kPer];
 #pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) {
-      const uint32_t ws[4] = {vw[k].x, vw[k].y, vw[k].z, vw[k].w};
+      for (int k = 0; k < kPer; ++k) {
+        const int i = base + tid + k * kClsThreads;
+        const int c = kt * kPfCells + i / per_row;
+        vw[k] = make_uint4(0u, 0u, 0u, 0u);
+        kw[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < n_chunk && c < p.N) {
+          vw[k] = __ldg(reinterpret_cast<const uint4*>(vbase + (int64_t)c * p.kv_sc) + (i % per_row));
+          if (p.kn2) kw[k] = __ldg(reinterpret_cast<const uint4*>(kbase + (int64_t)c * p.kv_sc) + (i % per_row));
+        }
+      }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) bad |= ((ws[q] & e_lo) == e_lo) | (((ws[q] >> 16) & e_lo) == e_lo);
+      for (int k = 0; k < kPer; ++k) {
+        const uint32_t ws[4] = {vw[k].x, vw[k].y, vw[k].z, vw[k].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) bad |= ((ws[q] & e_lo) == e_lo) | (((ws[q] >> 16) & e_lo) == e_lo);
+      }
+      if (p.kn2) {
+        // the per_row chunks of one cell sit in per_row consecutive lanes
+        // (per_row divides 32) or, at head dim 256, in one warp's 32 lanes
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+          const uint32_t ws[4] = {kw[k].x, kw[k].y, kw[k].z, kw[k].w};
+          float ss = 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float lo, hi;
+            if (p.kv_type == ATTN_BF16) {
+              lo = __uint_as_float(ws[q] << 16);
+              hi = __uint_as_float(ws[q] & 0xffff0000u);
+            } else {
+              lo = __half2float(__ushort_as_half((unsigned short)(ws[q] & 0xffffu)));
+              hi = __half2float(__ushort_as_half((unsigned short)(ws[q] >> 16)));
+            }
+            ss = fmaf(lo, lo, ss);
+            ss = fmaf(hi, hi, ss);
+          }
+          for (int o = min(per_row, 32) / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          mx = fmax_nan(mx, ss);
+        }
+      }
     }
     const int any_bad = __syncthreads_or(bad ? 1 : 0);
     if (tid == 0) p.vbad[(int64_t)kt * p.Hkv + g] = any_bad ? 1 : 0;
     if (p.kn2) {
-      // max over the tile's cells of |k_c|^2 (NaN-propagating: a non-finite K
-      // makes the bound fail)
-      float mx = 0.f;
-#pragma unroll
-      for (int k = 0; k < kMaxPer; ++k) {
-        const uint32_t ws[4] = {kw[k].x, kw[k].y, kw[k].z, kw[k].w};
-        float ss = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float lo, hi;
-          if (p.kv_type == ATTN_BF16) {
-            lo = __uint_as_float(ws[q] << 16);
-            hi = __uint_as_float(ws[q] & 0xffff0000u);
-          } else {
-            lo = __half2float(__ushort_as_half((unsigned short)(ws[q] & 0xffffu)));
-            hi = __half2float(__ushort_as_half((unsigned short)(ws[q] >> 16)));
-          }
-          ss = fmaf(lo, lo, ss);
-          ss = fmaf(hi, hi, ss);
-        }
-        for (int o = per_row / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        mx = fmax_nan(mx, ss);
-      }
       for (int o = 16; o > 0; o >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (lane == 0) wmax[warp] = mx;
       __syncthreads();
@@ -242,6 +244,21 @@ __global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPl
         p.kn2[(int64_t)kt * p.Hkv + g] = m;
       }
     }
+}
+
+// Blocks b < n_rt * n_kt classify tile b; the blocks after them scan one
+// (cell tile, KV head) each.
+__global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPlan p) {
+  pdl_launch_dependents();   // the prefill kernel may start its prologue
+  __shared__ int4 rows_sh[kPfRows];
+  __shared__ float wmax[kClsThreads / 32];
+  const int64_t b = blockIdx.x;
+  const int64_t n_cls = (int64_t)p.n_rt * p.n_kt;
+  if (b < n_cls) {
+    pf_classify_tile(p, b, rows_sh);
+  } else {
+    const int64_t vb = b - n_cls;
+    pf_scan_tile(p, (int)(vb / p.Hkv), (int)(vb % p.Hkv), wmax);
   }
 }
 
@@ -253,10 +270,13 @@ template <int D>
 struct PfLayout {
   static constexpr int BOX = 128 * 128;                  // one TMA box: 128 rows x 128 B (64 values)
   static constexpr int TILE = kPfRows * D * 2;           // a Q, K or V tile: D/64 boxes
-  static constexpr int NK = D == 64 ? 3 : 2;             // K ring stages (one tile each)
-  static constexpr int NV = D == 64 ? 4 : 3;             // V ring stages
-  static constexpr int OFF_Q = 0;                        // [2 slots][TILE]
-  static constexpr int OFF_K = OFF_Q + 2 * TILE;         // [NK][TILE]
+  // q heads per CTA (head slots): S and O of a head take 128 + D tensor-memory
+  // columns, so two heads fit the 512 columns up to head dim 128, one at 256
+  static constexpr int HPC = D <= 128 ? 2 : 1;
+  static constexpr int NK = D == 64 ? 3 : D == 128 ? 2 : 1;   // K ring stages (one tile each)
+  static constexpr int NV = D == 64 ? 4 : D == 128 ? 3 : 1;   // V ring stages
+  static constexpr int OFF_Q = 0;                        // [HPC slots][TILE]
+  static constexpr int OFF_K = OFF_Q + HPC * TILE;       // [NK][TILE]
   static constexpr int OFF_V = OFF_K + NK * TILE;        // [NV][TILE]
   static constexpr int OFF_BAR = OFF_V + NV * TILE;
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
@@ -275,15 +295,11 @@ struct PfLayout {
   static constexpr int HIGH_REGS = 224;
   static_assert(128 * LOW_REGS + 256 * HIGH_REGS <= THREADS * LAUNCH_REGS, "register split");
   static_assert(THREADS * LAUNCH_REGS <= 65536, "launch registers");
-  static constexpr uint32_t TMEM_COLS = 512;             // S0, S1 (128 each), O0, O1 (D each)
-  static_assert(2 * 128 + 2 * D <= (int)TMEM_COLS, "TMEM columns");
+  static constexpr uint32_t TMEM_COLS = 512;             // S_s at 128 s, O_s at 256 + D s
+  static_assert(HPC * 128 <= 256 && 256 + HPC * D <= (int)TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
-__device__ __forceinline__ unsigned char* pf_align1024(unsigned char* p) {
-  const uint32_t a = smem_u32(p);
-  return p + (((a + 1023u) & ~1023u) - a);
-}
 
 // K and V rings: the i-th K (or V) tile the CTA loads goes to stage i % NK
 // (i % NV); its "full" barrier completes phase i / NK for it, and the stage's
@@ -629,6 +645,55 @@ __device__ __forceinline__ void pf_store32(const OutSpec& o, int64_t i0, const f
   }
 }
 
+// Bound path (bf16 P only): one pass from the raw dot products of one
+// thread's row of a full or bits tile to P.  The caller has bounded every
+// logit of the tile by |scale| |q| max|k| plus the ALiBi ramp's largest value
+// and moved the running max m to that bound when it grew by more than ln 256,
+// so no per-cell max is needed (the weights stay <= 256; m only serves as the
+// common reference of l and O, and bf16 keeps the full float exponent range
+// for weights far below 1).  With log2(e) folded into the constants:
+//   a_i = s_i (bsc + w (b3 + w (b5 + w (b7 [+ w b9])))) + L (ramp_i - m),  w = s_i^2,
+// the softcap's odd series through u^DEG (DEG 0: no softcap), then
+// p_i = 2^a_i.  The ramp is L (C + slope i - m) = rbase + (8 mb) ls + rq[i % 8]
+// for block mb of 8 cells (one rounding per block, none carried along the
+// row).  Cells whose bit in vis is clear (bits tiles) get p = 0.  Returns the
+// sum of the p_i.
+template <int DEG, bool ALIBI, bool BITS>
+__device__ __forceinline__ float pf_tile_bound(const uint32_t* raw, uint32_t* pk, const PrefillPlan& p, float ls,
+                                               float rbase, const uint32_t* vis) {
+  const float2 B9 = f2(p.b9), B7 = f2(p.b7), B5 = f2(p.b5), B3 = f2(p.b3), BS = f2(p.bsc);
+  float2 RQ[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) RQ[k] = ALIBI ? f2(ls * (float)(2 * k), ls * (float)(2 * k + 1)) : f2(0.f);
+  float2 acc[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
+#pragma unroll
+  for (int mb = 0; mb < kPfCells / 8; ++mb) {
+    const float2 RB = f2(ALIBI ? fmaf(8.f * ls, (float)mb, rbase) : rbase);
+    const uint32_t vw = BITS ? (vis[mb >> 2] >> ((mb & 3) * 8)) : 0xffu;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = mb * 8 + 2 * k;
+      const float2 sv = f2(__uint_as_float(raw[i]), __uint_as_float(raw[i + 1]));
+      float2 t = BS;
+      if (DEG > 0) {
+        const float2 w = mul2(sv, sv);
+        float2 h = DEG == 9 ? fma2(w, fma2(w, fma2(w, B9, B7), B5), B3) : fma2(w, fma2(w, B7, B5), B3);
+        t = fma2(w, h, BS);
+      }
+      float2 a = fma2(sv, t, ALIBI ? add2(RB, RQ[k]) : RB);
+      if (BITS) {
+        a.x = ((vw >> (2 * k)) & 1u) ? a.x : neg_inf();
+        a.y = ((vw >> (2 * k + 1)) & 1u) ? a.y : neg_inf();
+      }
+      const float p0 = ex2(a.x), p1 = ex2(a.y);
+      acc[k] = add2(acc[k], f2(p0, p1));
+      pk[i / 2] = pf_pack<__nv_bfloat16>(p0, p1);
+    }
+  }
+  const float2 s = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+  return s.x + s.y;
+}
+
 // Lazy rescaling of the running state (m, l) by the tile max mt, then the
 // weights p_i = 2^((x_i + off_m) log2 e - m log2 e) of one row of a tile, their
 // sum into l, and P packed to 16 bits.  Block m of 8 cells adds the offset
@@ -750,7 +815,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     const int code = tiles.code(kt);
     if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p, abort_flag)) { ok = false; break; }
     tc_fence_after();
-    if (j == 0 && cap && p.kn2) {
+    if (j == 0 && p.kn2) {
       // the Q tile is resident (its load completed before the first S)
       if (!pf_wait_warp(B.q_full, 0u, p, abort_flag)) { ok = false; break; }
       const unsigned char* Qs = sm + L::OFF_Q + slot * L::TILE;
@@ -782,6 +847,75 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     const bool bits_tile = tiles.bits(kt);
     bool fast = (code == kTileFull || bits_tile) && (!cap || p.cap_raw) &&
                 (al == 0 || (al == 1 && !tiles.late(kt)));
+    bool done = false;
+    if constexpr (Storage<KT>::kDtype == ATTN_BF16) {
+      if (fast && p.kn2) {
+        // Bound path: every row's logits bounded by |scale| |q| max|k| (the
+        // softcap never increases |u|) plus the ALiBi ramp at the row's
+        // nearest visible cell of the tile; |scale| |q| max|k| <= 30 keeps the
+        // bound within 60 of the true max, so visible weights never underflow.
+        // The softcap series of degree 7 where |u| <= c / 3 for every row of
+        // the warp (truncation below 1e-6 c), degree 9 where |u| <= 0.4 c
+        // (below 3.7e-7 c).
+        const float qk2 = qn2 * __ldg(p.kn2 + (int64_t)kt * p.Hkv + tiles.g);
+        int deg = -1;
+        if (cap) deg = __all_sync(0xffffffffu, qk2 <= p.bound7) ? 7 : __all_sync(0xffffffffu, qk2 <= p.bound9) ? 9 : -1;
+        else deg = __all_sync(0xffffffffu, qk2 <= p.nc_lim2) ? 0 : -1;
+        if (deg >= 0) {
+          uint32_t raw[kPfCells];
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, raw + c4 * 32);
+          // visible cells of this row in the tile: all (full) or the stored bits
+          int i_lo = 0, i_hi = kPfCells - 1;
+          if (bits_tile) {
+            const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
+                                          p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_t) << 2)))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            vis[0] = bw.x; vis[1] = bw.y; vis[2] = bw.z; vis[3] = bw.w;
+            i_hi = vis[3] ? 96 + 31 - __clz(vis[3]) : vis[2] ? 64 + 31 - __clz(vis[2])
+                 : vis[1] ? 32 + 31 - __clz(vis[1]) : vis[0] ? 31 - __clz(vis[0]) : -1;
+            i_lo = vis[0] ? __ffs(vis[0]) - 1 : vis[1] ? 32 + __ffs(vis[1]) - 1
+                 : vis[2] ? 64 + __ffs(vis[2]) - 1 : vis[3] ? 96 + __ffs(vis[3]) - 1 : -1;
+          }
+          const float slope = -nslope, C = nslope * A;
+          // ramp C + slope i over the visible cells: largest at i_hi (slope >= 0) or i_lo
+          const float ramp_max = al == 1 ? fmaf(slope >= 0.f ? (float)i_hi : (float)i_lo, slope, C) : 0.f;
+          const float Mt = fabsf(scale) * sqrtf(qk2) + ramp_max;
+          constexpr float kLazy = 5.545177444479562f;   // ln 256
+          // a row that sees no cell of the tile leaves its state alone (a row
+          // that never sees a cell keeps m = -inf and is written as +0)
+          need = i_hi >= 0 && !(Mt <= m + kLazy);
+          factor = 1.f;
+          if (need) {
+            factor = ex2((m - Mt) * kLog2e);   // 0 when m was -inf
+            l *= factor;
+            m = Mt;
+            mneg2 = -m * kLog2e;
+          }
+          const float rbase = ((al == 1 ? C : 0.f) - m) * kLog2e, lsl = slope * kLog2e;
+          tmem_wait_ld();
+          float ts;
+          if (al == 1) {
+            if (bits_tile) ts = deg == 7 ? pf_tile_bound<7, true, true>(raw, pk, p, lsl, rbase, vis)
+                              : deg == 9 ? pf_tile_bound<9, true, true>(raw, pk, p, lsl, rbase, vis)
+                                         : pf_tile_bound<0, true, true>(raw, pk, p, lsl, rbase, vis);
+            else ts = deg == 7 ? pf_tile_bound<7, true, false>(raw, pk, p, lsl, rbase, vis)
+                      : deg == 9 ? pf_tile_bound<9, true, false>(raw, pk, p, lsl, rbase, vis)
+                                 : pf_tile_bound<0, true, false>(raw, pk, p, lsl, rbase, vis);
+          } else {
+            if (bits_tile) ts = deg == 7 ? pf_tile_bound<7, false, true>(raw, pk, p, lsl, rbase, vis)
+                              : deg == 9 ? pf_tile_bound<9, false, true>(raw, pk, p, lsl, rbase, vis)
+                                         : pf_tile_bound<0, false, true>(raw, pk, p, lsl, rbase, vis);
+            else ts = deg == 7 ? pf_tile_bound<7, false, false>(raw, pk, p, lsl, rbase, vis)
+                      : deg == 9 ? pf_tile_bound<9, false, false>(raw, pk, p, lsl, rbase, vis)
+                                 : pf_tile_bound<0, false, false>(raw, pk, p, lsl, rbase, vis);
+          }
+          l += i_hi >= 0 ? ts : 0.f;
+          done = true;
+          fast = false;
+        }
+      }
+    }
     if (fast) {
       uint32_t raw[kPfCells];
 #pragma unroll
@@ -818,7 +952,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
         pf_weights<KT>(x, boff, bstep, mt, m, l, mneg2, pk, need, factor);
       }
     }
-    if (!fast) {
+    if (!fast && !done) {
       const int32_t* cpos = p.f.cell_pos ? p.f.cell_pos + c0 : nullptr;
       // full tiles: ALiBi in the transform; mixed tiles with explicit
       // positions: in the visibility pass (cell_pos may end inside the tile)
@@ -941,9 +1075,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int rt = p.n_rt - 1 - (int)(blockIdx.x / per_rt);
   const int g = (int)(blockIdx.x % per_rt) / p.n_pairs;
   const int pair = (int)(blockIdx.x % per_rt) % p.n_pairs;
-  const int h0 = g * p.G + 2 * pair;
-  const bool two = 2 * pair + 1 < p.G;
-  const int n_slots = two ? 2 : 1;
+  const int h0 = g * p.G + L::HPC * pair;
+  const int n_slots = min(L::HPC, p.G - L::HPC * pair);
 
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 1);
@@ -1118,6 +1251,9 @@ cudaError_t launch_prefill(const PrefillPlan& p, const CUtensorMap& tmQ, const C
   if (p.D == 64)
     return bf ? launch_prefill_t<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, stream, after_classify)
               : launch_prefill_t<__half, 64>(p, tmQ, tmK, tmV, stream, after_classify);
+  if (p.D == 256)
+    return bf ? launch_prefill_t<__nv_bfloat16, 256>(p, tmQ, tmK, tmV, stream, after_classify)
+              : launch_prefill_t<__half, 256>(p, tmQ, tmK, tmV, stream, after_classify);
   return bf ? launch_prefill_t<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, stream, after_classify)
             : launch_prefill_t<__half, 128>(p, tmQ, tmK, tmV, stream, after_classify);
 }

@@ -28,10 +28,12 @@
  *                  PR #910).  QK^T and PV run on the tensor cores in tiles of
  *                  128 rows x 128 cells; P is rounded to the K/V dtype before
  *                  PV.  Supported: K/V and Q in F16 or BF16 (same dtype),
- *                  head_dim 64 or 128, Q 16-byte aligned with strides that are
- *                  multiples of 16 bytes; any out dtype.  n_slices, max_row_len
- *                  and grid_order are ignored.  Workspace: one byte per
- *                  (128-row tile, 128-cell tile) and per (cell tile, KV head).
+ *                  head_dim 64, 128 or 256, Q 16-byte aligned with strides
+ *                  that are multiples of 16 bytes; any out dtype.  n_slices,
+ *                  max_row_len and grid_order are ignored.  Workspace: one
+ *                  byte per (128-row tile, 128-cell tile) and per (cell tile,
+ *                  KV head), plus the visibility bits of every tile when a
+ *                  mask is given.
  *
  * Unified caches.  When cell_seq/row_seq are given (several sequences'
  * cells interleaved in one cache, strix-llama.cpp PR #115 "Isolation"), the
@@ -101,6 +103,10 @@
  * dequantized K/V.  Strides stay in elements (= bytes).  k_scale, v_scale:
  * F32 device arrays, non-NULL for a quantized cache with n_cells > 0 and NULL
  * otherwise; scale_stride_cell >= n_head_kv.  Q and out are never quantized.
+ * With n_slices == 0, Q in BF16 or F16 (16-byte aligned, strides multiples of
+ * 8 elements), head_dim 128 or 256 and at most 8 query heads per KV head, the
+ * codes run on the tensor cores (widened to f16 in registers, which is exact);
+ * other shapes and forced slice counts run on the CUDA cores.
  * attn_selected and attn_prefill refuse quantized caches (ATTN_ERR_UNSUPPORTED).
  */
 #ifndef ATTN_B200_H

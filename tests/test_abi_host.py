@@ -154,14 +154,22 @@ def test_empty_problem_is_ok(lib):
 
 
 def test_quantized_decode_slice_plan(lib):
-    """e4m3/int8 caches take 2048-cell slices: 8192-cell rows -> 4 slices,
-    R * Hq * 4 partial records of D + 2 floats."""
+    """e4m3/int8 caches on the CUDA-core grid kernel (here: an F32 query) take
+    2048-cell slices: 8192-cell rows -> 4 slices, R * Hq * 4 partial records
+    of D + 2 floats.  With a BF16 query the balanced tensor-core kernel takes
+    them instead: the row tile prefix and one record per warp and per
+    (row, KV head)."""
     a = _args(n_rows=16, n_head_q=32, n_head_kv=8, n_cells=131072, max_row_len=8192,
-              kv_type=A.ATTN_FP8_E4M3, kv_stride_cell=8 * 128, kv_stride_head=128)
+              kv_type=A.ATTN_FP8_E4M3, kv_stride_cell=8 * 128, kv_stride_head=128, q_type=A.ATTN_F32)
     a.k_scale, a.v_scale, a.scale_stride_cell = 0x60000, 0x70000, 8
     ws = lib.attn_workspace_size(ctypes.byref(a), A.OP_DECODE, 0)
     slots = 16 * 32 * 4
     assert ws == (slots * 128 * 4 + 255) // 256 * 256 + (slots * 2 * 4 + 255) // 256 * 256
+    a.q_type = A.ATTN_BF16
+    ws_tc = lib.attn_workspace_size(ctypes.byref(a), A.OP_DECODE, 0)
+    tiles = (17 * 8 + 255) // 256 * 256
+    records = (ws_tc - tiles) // ((128 + 2) * 4)   # (W + R * Hkv) * G, up to the 256-byte padding
+    assert records >= 16 * 8 * 4 and ws_tc != ws
     a.n_slices = 3                 # a forced count still wins
     ws = lib.attn_workspace_size(ctypes.byref(a), A.OP_DECODE, 0)
     slots = 16 * 32 * 3

@@ -27,7 +27,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("kv", [torch.float16, torch.bfloat16])
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 3, 8])
 def test_dtype_dim_group_sweep(cuda_lib, kv, D, G):
     p = W.random_prefill(100 + D + G + (0 if kv == torch.float16 else 7), R=130, Hq=2 * G, Hkv=2, D=D,
