@@ -362,13 +362,17 @@ __device__ __forceinline__ bool pf_wait_warp(uint64_t* bar, uint32_t parity, con
 // S (TMEM, 128 x 128 f32) = Q (128 x D) . K (128 x D)^T; both operands K-major
 // 128-byte-swizzled boxes of 64 columns.  One MMA per 16 columns of D: inside a
 // box the start address advances by 32 bytes, across boxes by one box.
+// The descriptors come in prebuilt: a descriptor's start-address field is
+// its low 14 bits (byte address >> 4), so the descriptor of base + off is
+// desc(base) + (off >> 4) -- no carry, shared-memory addresses stay below
+// 2^18 bytes.  One thread issues all MMAs while two softmax warps share its
+// scheduler, so every instruction saved here shortens the tensor core's wait.
 template <int D>
-__device__ __forceinline__ void pf_issue_s(uint32_t d_tmem, uint32_t q_base, uint32_t k_base, uint32_t idesc) {
+__device__ __forceinline__ void pf_issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc, uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (uint32_t)(kk >> 2) * PfLayout<D>::BOX + (uint32_t)(kk & 3) * 32u;
-    umma_ss(d_tmem, umma_desc_sw128(q_base + off, 16, 1024), umma_desc_sw128(k_base + off, 16, 1024), idesc,
-            kk > 0 ? 1u : 0u);
+    const uint64_t off = (uint64_t)(((kk >> 2) * PfLayout<D>::BOX + (kk & 3) * 32) >> 4);
+    umma_ss(d_tmem, q_desc + off, k_desc + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -378,12 +382,12 @@ __device__ __forceinline__ void pf_issue_s(uint32_t d_tmem, uint32_t q_base, uin
 // cells x D, D contiguous) is MN-major: its 8-cell groups are 1024 bytes apart
 // (SBO) and its 64-column boxes one box apart (LBO).
 template <int D>
-__device__ __forceinline__ void pf_issue_pv_ts(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_base, uint32_t idesc,
+__device__ __forceinline__ void pf_issue_pv_ts(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, uint32_t idesc,
                                                bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < kPfCells / 16; ++kk)
-    umma_ts(d_tmem, p_tmem + (uint32_t)kk * 8u, umma_desc_sw128(v_base + (uint32_t)kk * 2048u, PfLayout<D>::BOX, 1024),
-            idesc, (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, p_tmem + (uint32_t)kk * 8u, v_desc + (uint64_t)((kk * 2048) >> 4), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Cell tiles of one row tile, skipping the empty ones, from the LAST to the
@@ -1159,9 +1163,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr int bf = Storage<KT>::kDtype == ATTN_BF16 ? 1 : 0;
       constexpr uint32_t idS = umma_idesc_f16(kPfRows, kPfCells, bf, 0, 0);
       constexpr uint32_t idO = umma_idesc_f16(kPfRows, D, bf, 0, 1);
-      const uint32_t q_addr = smem_u32(sm + L::OFF_Q);
-      const uint32_t k_addr = smem_u32(sm + L::OFF_K);
-      const uint32_t v_addr = smem_u32(sm + L::OFF_V);
+      // descriptors of slot 0's Q, stage 0's K (K-major, 128-byte swizzle) and
+      // stage 0's V (MN-major); other slots / stages are whole tiles further
+      const uint64_t q_desc = umma_desc_sw128(smem_u32(sm + L::OFF_Q), 16, 1024);
+      const uint64_t k_desc = umma_desc_sw128(smem_u32(sm + L::OFF_K), 16, 1024);
+      const uint64_t v_desc = umma_desc_sw128(smem_u32(sm + L::OFF_V), L::BOX, 1024);
+      constexpr uint64_t kTileDesc = (uint64_t)(L::TILE >> 4);
       int kt = tiles.first();
       bool ok = kt >= 0;
       if (ok) {
@@ -1169,7 +1176,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (ok) {
           tc_fence_after();
           for (int s = 0; s < n_slots; ++s) {
-            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, k_addr, idS);
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_desc + (uint64_t)s * kTileDesc, k_desc, idS);
             umma_commit(&B.s_full[s]);
           }
           umma_commit(&B.k_empty[0]);
@@ -1187,13 +1194,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (s == 0 && !pf_wait(&B.v_full[stV], pf_phase<NV>(j), p, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if (pv_mma)
-            pf_issue_pv_ts<D>(tmem + 256u + (uint32_t)s * D, tmem + (uint32_t)s * 128u, v_addr + stV * L::TILE,
-                              idO, j > 0);
+            pf_issue_pv_ts<D>(tmem + 256u + (uint32_t)s * D, tmem + (uint32_t)s * 128u,
+                              v_desc + (uint64_t)stV * kTileDesc, idO, j > 0);
           umma_commit(&B.pv_done[s]);
           if (has_next) {
             if (s == 0 && !pf_wait(&B.k_full[stK], pf_phase<NK>(j + 1), p, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_addr + s * L::TILE, k_addr + stK * L::TILE, idS);
+            pf_issue_s<D>(tmem + (uint32_t)s * 128u, q_desc + (uint64_t)s * kTileDesc, k_desc + (uint64_t)stK * kTileDesc,
+                          idS);
             umma_commit(&B.s_full[s]);
             if (s == n_slots - 1) umma_commit(&B.k_empty[stK]);
           }

@@ -198,8 +198,36 @@ def cpu_baseline():
         if time.perf_counter() - t0 > 10.0:
             break
     dt = (time.perf_counter() - t0) / n
+    # one thread, rows 0-1 (the 1-thread figure)
+    rate1, _, n1 = _oracle_rate(p, [0, 1], algorithmic_bytes, budget_s=2.0, threads=1)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": min(cores, p.n_rows), "kind": "oracle",
-            "sample": f"the full 16-row batch, {n} repetitions (~10 s), one thread per row"}
+            "sample": f"the full 16-row batch, {n} repetitions (~10 s), one thread per row",
+            "value_1thread": rate1 / 1e9, "sample_1thread": f"rows 0-1 on one thread, {n1} repetitions (~2 s)"}
+
+
+def _oracle_rate(p, rows, amount_fn, budget_s=2.0, threads=0):
+    """The FP64 oracle as it stands on rows `rows` of problem p, repeated for
+    about budget_s on the host cores (one thread per row, or `threads`);
+    returns (amount_fn(rows) per second, threads used, repetitions)."""
+    import oracle
+    sub = p.row_subset(rows)
+    prep = oracle.Prepared(sub)
+    n_thr = threads or min(os.cpu_count() or 1, len(rows))
+    prep.run(n_threads=n_thr)
+    t0, n = time.perf_counter(), 0
+    while True:
+        prep.run(n_threads=n_thr)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return amount_fn(sub) / dt, n_thr, n
+
+
+def _part_baseline(p, rows, amount_fn, unit, scale, what):
+    rate, thr, n = _oracle_rate(p, rows, amount_fn)
+    return {"value": rate / scale, "unit": unit, "cores": thr, "kind": "oracle",
+            "sample": f"{what}, {n} repetitions (~2 s)"}
 
 
 def run_ours(args, rank, world, local):
@@ -271,7 +299,8 @@ def run_ours(args, rank, world, local):
     traffic = _recorded_traffic("decode_stream_kernel")
 
     e2e = run_e2e(args, sets, stream)
-    parts = None if args.no_parts else run_parts(args, rank, dev, stream)
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    parts = None if args.no_parts else run_parts(args, rank, dev, stream, with_cpu)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
@@ -294,6 +323,17 @@ def run_ours(args, rank, world, local):
         line["gpu_launches"] += sum(p_["gpu_launches"] for p_ in parts.values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
+    # one compact entry per workload, last on the line
+    summ = {"gqa_decode": f"{value:.0f} GB/s whole step, kernel {achieved:.0f} GB/s = {achieved / hbm_peak:.3f} of HBM"}
+    for name, pt in (parts or {}).items():
+        r = pt.get("roofline")
+        s_ = f"{pt['value']:.4g} {pt['unit'].split(' (')[0]}"
+        if r:
+            s_ += f", kernel {r['achieved']:.4g} {r['unit']} = {r['frac']:.3f} of {r['bound']}"
+        if "cpu_baseline" in pt:
+            s_ += f"; oracle {pt['cpu_baseline']['value']:.3g} {pt['cpu_baseline']['unit']} on {pt['cpu_baseline']['cores']} cores"
+        summ[name] = s_
+    line["summary"] = summ
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -362,13 +402,46 @@ def prefill_flops(p) -> int:
     return 4 * p.head_dim * vis * p.n_head_q
 
 
-def run_parts(args, rank, dev, stream):
-    """The selected-key and causal-prefill workloads, each timed per call
-    (L2 flushed before every call), with the roofline of its main kernel."""
+def run_parts(args, rank, dev, stream, with_cpu=False):
+    """The other workloads (tiny decode, selected-key, causal prefill,
+    draft-tree rows, e4m3 decode, the semantics sweep), each timed per call
+    (L2 flushed before every call), with the roofline of its main kernel and,
+    with_cpu, the FP64 oracle timed beside it on a bounded sample."""
     hbm_peak, tc_peak, peak_kind = _peaks()
     flush = _L2Flush(dev)
     n = max(3, min(args.steps, 20))
     parts = {}
+
+    # tiny decode (1 row, 4 q heads over 1 KV head, D 64, 128 FP32 keys, 4
+    # slices): a latency case -- the mean time of one call over back-to-back
+    # calls (inputs resident, no flush: they are 64 KB)
+    p = W.tiny_decode()
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    ta = A.make_args(q, k, v, out, **kw)
+    ws = torch.empty(max(A.workspace_size(ta, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+    for _ in range(20):
+        A.attn_decode_args(ta, ws=ws, stream=stream)
+    reps = 200
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        A.attn_decode_args(ta, ws=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    tiny_bytes = 2 * p.k.numel() * 4 + p.q.numel() * 4 + p.n_rows * p.n_head_q * p.head_dim * 4
+    parts["tiny_decode"] = {
+        "workload": "tiny_decode: 1 row, Hq 4 / Hkv 1, D 64, 128 FP32 keys, 4 forced slices, f32 out",
+        "value": us, "unit": "us per call (latency; back-to-back calls)", "higher_is_better": False,
+        "rows_per_s": 1e6 / us, "GBs": tiny_bytes / (us * 1e-6) / 1e9, "calls": reps,
+        "gpu_launches": 2 * reps,   # (rows, heads, slices) grid kernel + split_k_reduce
+    }
+    if with_cpu:
+        rate, thr, nrep = _oracle_rate(p, [0], lambda s_: 1, threads=1)
+        parts["tiny_decode"]["cpu_baseline"] = {"value": 1e6 / rate, "unit": "us per call", "cores": 1,
+                                                "kind": "oracle", "sample": f"the whole call, {nrep} repetitions"}
+    del q, k, v, out, ta, ws, kw
 
     # maskless selected-key: 2048 rows, GQA 12, D 256, fp16 cache of 32768 cells
     p = W.selected_prefill()
@@ -394,6 +467,9 @@ def run_parts(args, rank, dev, stream):
                      "kernel_ms": main, "algorithmic_bytes": nbytes,
                      "peak_kind": f"{peak_kind} hbm_gbs (burst copy); gathered rows are mostly L2 hits"},
     }
+    if with_cpu:
+        parts["selected"]["cpu_baseline"] = _part_baseline(p, list(range(0, 2048, 128)), selected_bytes, "GB/s",
+                                                           1e9, "16 of the 2048 rows (every 128th)")
     del q, k, v, out, sel, sa, ws, kw
 
     # causal prefill: 2048 rows over 14048 cells, Hq 64 / Hkv 8, D 128, bf16
@@ -418,6 +494,9 @@ def run_parts(args, rank, dev, stream):
                      "kernel_ms": main, "algorithmic_flops": flops,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS)"},
     }
+    if with_cpu:
+        parts["prefill"]["cpu_baseline"] = _part_baseline(p, [128 * i + 64 for i in range(16)], prefill_flops,
+                                                          "TFLOP/s", 1e12, "16 of the 2048 rows (one per row tile)")
     del q, k, v, out, pa, ws, kw
 
     # draft-tree decode rows: 16 nodes of a binary draft tree over 130856 keys
@@ -460,6 +539,9 @@ def run_parts(args, rank, dev, stream):
                      "algorithmic_bytes": tbytes,
                      "peak_kind": f"{peak_kind} hbm_gbs (burst copy); each row streams the shared prefix"},
     }
+    if with_cpu:
+        parts["tree_decode"]["cpu_baseline"] = _part_baseline(
+            p, list(range(p.n_rows)), lambda s_: tbytes, "GB/s", 1e9, "all 16 rows")
     del q, k, v, out, ta, ws, kw, tmask
 
     # quantized GQA decode: the decode batch's shape (16 rows, lengths U[1024,
@@ -485,9 +567,13 @@ def run_parts(args, rank, dev, stream):
         "gpu_launches": (2 if qws_n > 0 else 1) * n,   # slice kernel (+ split_k_reduce)
         "roofline": {"bound": "hbm", "achieved": qbytes / (main * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": qbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None, "kernel_ms": main,
-                     "algorithmic_bytes": qbytes, "kernel": "decode_slice_kernel<e4m3> (+ combine_kernel)",
+                     "algorithmic_bytes": qbytes,
+                     "kernel": "decode_stream_kernel<e4m3> (codes widened to f16 for the tensor cores) + combine_kernel",
                      "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
     }
+    if with_cpu:
+        parts["fp8_decode"]["cpu_baseline"] = _part_baseline(
+            p, list(range(p.n_rows)), lambda s_: qbytes, "GB/s", 1e9, "all 16 rows")
     del q, k, v, out, qa, ws, kw
 
     # semantics sweep: unified fp16 cache of 8 interleaved sequences, 256 rows,
@@ -520,6 +606,10 @@ def run_parts(args, rank, dev, stream):
                          "kernel_ms": main, "algorithmic_bytes": nbytes,
                          "peak_kind": f"{peak_kind} hbm_gbs (burst copy); semantics case, no target"},
         }
+    if with_cpu:
+        base = _part_baseline(p, list(range(p.n_rows)), lambda s_: nbytes, "GB/s", 1e9, "all 256 rows")
+        parts["semantics_decode"]["cpu_baseline"] = base
+        parts["semantics_prefill"]["cpu_baseline"] = base
     return parts
 
 
