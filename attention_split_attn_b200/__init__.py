@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
 
 ATTN_F32, ATTN_F16, ATTN_BF16, ATTN_FP8_E4M3, ATTN_I8 = 0, 1, 2, 3, 4
-OP_DECODE, OP_SELECTED, OP_PREFILL = 0, 1, 2
+OP_DECODE, OP_SELECTED, OP_PREFILL, OP_SELECTED_MASKED = 0, 1, 2, 3
 STATUS = {0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED",
           -3: "ATTN_ERR_WORKSPACE", -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_DEVICE_TIMEOUT"}
 
@@ -33,7 +33,7 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
            "attn_prefill", "attn_decode_timed", "attn_selected_timed", "attn_prefill_timed",
-           "attn_decode_noalloc", "attn_tree_mask",
+           "attn_decode_noalloc", "attn_tree_mask", "attn_selected_masked", "attn_selected_masked_timed",
            "attn_check_device_status",
            "attn_strerror", "attn_last_error", "attn_abi_version")
 
@@ -111,6 +111,13 @@ def load_library():
             lib.attn_selected_timed.restype = ctypes.c_int32
             lib.attn_selected_timed.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
                                                 ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p * 3]
+            for name in ("attn_selected_masked",):
+                fn = getattr(lib, name)
+                fn.restype = ctypes.c_int32
+                fn.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            lib.attn_selected_masked_timed.restype = ctypes.c_int32
+            lib.attn_selected_masked_timed.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
+                                                       ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p * 3]
             lib.attn_tree_mask.restype = ctypes.c_int32
             lib.attn_tree_mask.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
@@ -323,6 +330,40 @@ def attn_selected_timed_args(args: AttnSelectedArgs, ws: Optional[torch.Tensor],
                                  0 if ws is None else ws.numel() * ws.element_size(),
                                  _stream_handle(stream), ev)
     _raise_if(st, "attn_selected_timed")
+
+
+def attn_selected_masked_args(args: AttnSelectedArgs, ws: Optional[torch.Tensor] = None, stream=None):
+    """The masked per-cell route of selected-key attention (per-cell mask + the
+    dense tensor-core pass; see include/attn.h) on a prepared AttnSelectedArgs."""
+    lib = load_library()
+    _raise_if(lib.attn_supports(ctypes.byref(args.base), OP_SELECTED_MASKED), "attn_supports")
+    need = int(lib.attn_workspace_size(ctypes.byref(args.base), OP_SELECTED_MASKED, args.n_sel))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = _workspace(need, dev, ws)
+    st = lib.attn_selected_masked(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
+    _raise_if(st, "attn_selected_masked")
+    return ws
+
+
+def attn_selected_masked_timed_args(args: AttnSelectedArgs, ws: Optional[torch.Tensor], events, stream=None):
+    """attn_selected_masked that also records three torch.cuda.Events (before
+    the mask kernel, after the tensor-core kernel, after the last kernel)."""
+    lib = load_library()
+    handles = [None if e is None else e.cuda_event for e in events]
+    if any(h == 0 for h in handles):
+        raise ValueError("record each torch.cuda.Event once before passing it (torch creates it lazily)")
+    ev = (ctypes.c_void_p * 3)(*handles)
+    st = lib.attn_selected_masked_timed(ctypes.byref(args), None if ws is None else ws.data_ptr(),
+                                        0 if ws is None else ws.numel() * ws.element_size(),
+                                        _stream_handle(stream), ev)
+    _raise_if(st, "attn_selected_masked_timed")
+
+
+def selected_masked_workspace_size(args: AttnSelectedArgs) -> int:
+    lib = load_library()
+    _raise_if(lib.attn_supports(ctypes.byref(args.base), OP_SELECTED_MASKED), "attn_supports")
+    return int(lib.attn_workspace_size(ctypes.byref(args.base), OP_SELECTED_MASKED, args.n_sel))
 
 
 def selected_workspace_size(args: AttnSelectedArgs) -> int:

@@ -384,18 +384,44 @@ int32_t check_prefill(const attn_args* a) {
   }
   const int64_t n_rt = ((int64_t)a->n_rows + kPfTile - 1) / kPfTile;
   const int G = a->n_head_q / a->n_head_kv;
-  const int64_t ctas = n_rt * a->n_head_kv * (a->head_dim <= 128 ? (G + 1) / 2 : G);
+  const int64_t ctas = 4 * n_rt * a->n_head_kv * (a->head_dim <= 128 ? (G + 1) / 2 : G);   // split parts included
   const int64_t n_kt = ((int64_t)a->n_cells + kPfTile - 1) / kPfTile;
   if (ctas > 0x7fffffffLL || n_rt * n_kt + n_kt * a->n_head_kv > 0x7fffffffLL)
     return fail(ATTN_ERR_UNSUPPORTED, "prefill: grid too large");
   return ATTN_OK;
 }
 
-struct PrefillWs {
-  size_t vbad_off, kn2_off, bits_off, total;
+// Work units of the tensor-core kernel: (row tile, KV head, q heads per CTA),
+// heaviest row tiles first.  The units of a last, partial wave over the SMs
+// (or every unit, when there are fewer units than SMs) are split into k
+// parts over their cell tiles, k = SMs / (those units) clamped to 2..4, so
+// the last wave holds shorter pieces; the parts' (m, l, O) are folded by the
+// last part to finish.
+struct PrefillSplit {
+  int64_t units, n_full, n_split;   // n_split units of k parts each
+  int32_t k;
+  int64_t ctas() const { return n_full + n_split * k; }
 };
 
-PrefillWs prefill_ws_layout(const attn_args* a) {
+PrefillSplit plan_prefill_split(const attn_args* a, int sms) {
+  PrefillSplit s{};
+  const int64_t n_rt = ((int64_t)a->n_rows + kPfTile - 1) / kPfTile;
+  const int G = a->n_head_q / a->n_head_kv;
+  s.units = n_rt * a->n_head_kv * (a->head_dim <= 128 ? (G + 1) / 2 : G);
+  const int64_t r = s.units > sms ? s.units % sms : s.units;
+  const int64_t k = r > 0 ? std::min<int64_t>(4, sms / r) : 1;
+  s.k = (int32_t)k;
+  s.n_split = k >= 2 ? r : 0;
+  s.n_full = s.units - s.n_split;
+  if (k < 2) s.k = 1;
+  return s;
+}
+
+struct PrefillWs {
+  size_t vbad_off, kn2_off, bits_off, cnt_off, po_off, pml_off, total;
+};
+
+PrefillWs prefill_ws_layout(const attn_args* a, const PrefillSplit& sp) {
   const size_t n_rt = ((size_t)a->n_rows + kPfTile - 1) / kPfTile;
   const size_t n_kt = ((size_t)a->n_cells + kPfTile - 1) / kPfTile;
   PrefillWs w;
@@ -404,7 +430,14 @@ PrefillWs prefill_ws_layout(const attn_args* a) {
   w.bits_off = w.kn2_off + align256(n_kt * a->n_head_kv * sizeof(float));
   // visibility bits of every tile when a mask is given (1/32 of the mask's size)
   const size_t bits = a->mask ? n_rt * n_kt * (size_t)kPfTile * 16 : 0;
-  w.total = w.bits_off + align256(bits);
+  w.cnt_off = w.bits_off + align256(bits);
+  // split units: a counter each, and per part and q head slot the 128 rows'
+  // unnormalised O [D] and (m, l)
+  const size_t hpc = a->head_dim <= 128 ? 2 : 1;
+  const size_t recs = (size_t)sp.n_split * (size_t)sp.k * hpc * kPfTile;
+  w.po_off = w.cnt_off + align256((size_t)sp.n_split * 2 * kPfTile * sizeof(int));   // per (unit, slot, row)
+  w.pml_off = w.po_off + align256(recs * a->head_dim * sizeof(float));
+  w.total = w.pml_off + align256(recs * 2 * sizeof(float));
   return w;
 }
 
@@ -528,11 +561,33 @@ const char* attn_strerror(int32_t s) {
 
 const char* attn_last_error(void) { return g_last_error.c_str(); }
 
+// ---- masked route of selected-key attention ----------------------------------------
+// The dense prefill arguments under which the masked route computes the
+// selected op: the selected arguments plus the per-cell mask (row stride a
+// multiple of 4 floats), no ranges, sequences or causal flag; positions as given.
+int64_t sel_mask_ld(const attn_args* b) { return ((int64_t)b->n_cells + 3) / 4 * 4; }
+attn_args sel_mask_args(const attn_args* b, float* mask) {
+  attn_args pa = *b;
+  pa.mask = mask;
+  pa.mask_stride_row = sel_mask_ld(b);
+  return pa;
+}
+size_t sel_mask_bytes(const attn_args* b) { return align256((size_t)b->n_rows * sel_mask_ld(b) * sizeof(float)); }
+
+int32_t check_selected_masked(const attn_args* b) {
+  int32_t st = check_selected_base(b);
+  if (st != ATTN_OK) return st;
+  // the dense route's own limits (the mask pointer only needs to be non-NULL and aligned here)
+  const attn_args pa = sel_mask_args(b, reinterpret_cast<float*>(static_cast<uintptr_t>(256)));
+  return check_prefill(&pa);
+}
+
 int32_t attn_supports(const attn_args* a, int32_t op) {
   switch (op) {
     case ATTN_OP_DECODE: return check_decode(a);
     case ATTN_OP_SELECTED: return check_selected_base(a);
     case ATTN_OP_PREFILL: return check_prefill(a);
+    case ATTN_OP_SELECTED_MASKED: return check_selected_masked(a);
     default: return fail(ATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
 }
@@ -547,7 +602,13 @@ size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
     case ATTN_OP_SELECTED:
       if (n_sel < 1 || n_sel > kMaxSel) return 0;
       return selected_ws_layout(a, n_sel, plan_selected(a, n_sel, sms)).total;
-    case ATTN_OP_PREFILL: return unified_route(a) ? unified_ws_bytes(a, sms) : prefill_ws_layout(a).total;
+    case ATTN_OP_PREFILL:
+      return unified_route(a) ? unified_ws_bytes(a, sms) : prefill_ws_layout(a, plan_prefill_split(a, sms)).total;
+    case ATTN_OP_SELECTED_MASKED: {
+      if (n_sel < 1 || n_sel > kMaxSel) return 0;
+      const attn_args pa = sel_mask_args(a, reinterpret_cast<float*>(static_cast<uintptr_t>(256)));
+      return sel_mask_bytes(a) + prefill_ws_layout(&pa, plan_prefill_split(&pa, sms)).total;
+    }
     default: return 0;
   }
 }
@@ -648,6 +709,39 @@ int32_t attn_selected(const attn_selected_args* a, void* ws, size_t ws_bytes, vo
   return attn_selected_timed(a, ws, ws_bytes, stream, nullptr);
 }
 
+int32_t attn_selected_masked(const attn_selected_args* a, void* ws, size_t ws_bytes, void* stream) {
+  return attn_selected_masked_timed(a, ws, ws_bytes, stream, nullptr);
+}
+
+int32_t attn_selected_masked_timed(const attn_selected_args* a, void* ws, size_t ws_bytes, void* stream,
+                                   void* const events[3]) {
+  if (!a) return fail(ATTN_ERR_INVALID_ARG, "args is NULL");
+  const attn_args* b = &a->base;
+  int32_t st = check_selected_masked(b);
+  if (st != ATTN_OK) return st;
+  if (a->n_sel < 1 || a->n_sel > kMaxSel) return fail(ATTN_ERR_UNSUPPORTED, "n_sel must be 1..%d", kMaxSel);
+  if (b->n_rows == 0) return ATTN_OK;
+  if (!a->sel) return fail(ATTN_ERR_INVALID_ARG, "sel is NULL");
+  if (a->sel_stride_row < a->n_sel) return fail(ATTN_ERR_INVALID_ARG, "sel_stride_row is smaller than n_sel");
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(ATTN_ERR_WORKSPACE, "the masked route needs a 256-byte aligned workspace");
+  const size_t mb = sel_mask_bytes(b);
+  if (ws_bytes < mb) return fail(ATTN_ERR_WORKSPACE, "the masked route needs %zu bytes for its mask", mb);
+  float* mask = static_cast<float*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  record_event(events, 0, s);
+  if (b->n_cells > 0) {
+    const cudaError_t e = launch_sel_mask(a->sel, a->sel_stride_row, a->n_sel, b->n_rows, b->n_cells, mask,
+                                          sel_mask_ld(b), s);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "selection mask launch: %s", cudaGetErrorString(e));
+  }
+  const attn_args pa = sel_mask_args(b, mask);
+  // the dense pass (its own workspace after the mask); the first event stays
+  // in front of the mask kernel
+  void* const ev2[3] = {nullptr, events ? events[1] : nullptr, events ? events[2] : nullptr};
+  return attn_prefill_timed(&pa, static_cast<char*>(ws) + mb, ws_bytes - mb, stream, events ? ev2 : nullptr);
+}
+
 int32_t attn_selected_timed(const attn_selected_args* a, void* ws, size_t ws_bytes, void* stream,
                             void* const events[3]) {
   if (!a) return fail(ATTN_ERR_INVALID_ARG, "args is NULL");
@@ -722,7 +816,8 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != ATTN_OK) return st;
   if (unified_route(a)) return run_unified(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), events, di);
-  const PrefillWs wl = prefill_ws_layout(a);
+  const PrefillSplit sp = plan_prefill_split(a, di->sms);
+  const PrefillWs wl = prefill_ws_layout(a, sp);
   if (wl.total > 0 && (ws == nullptr || ws_bytes < wl.total))
     return fail(ATTN_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", wl.total, ws_bytes);
   if (wl.total > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
@@ -761,6 +856,12 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   p.vbad = reinterpret_cast<uint8_t*>(wsb + wl.vbad_off);
   p.kn2 = reinterpret_cast<float*>(wsb + wl.kn2_off);
   p.bits = a->mask ? reinterpret_cast<uint32_t*>(wsb + wl.bits_off) : nullptr;
+  p.n_full = sp.n_full;
+  p.n_split = sp.n_split;
+  p.k_split = sp.k;
+  p.split_cnt = reinterpret_cast<int*>(wsb + wl.cnt_off);
+  p.part_o = reinterpret_cast<float*>(wsb + wl.po_off);
+  p.part_ml = reinterpret_cast<float*>(wsb + wl.pml_off);
   // Softcap polynomial: x = u + u w (k3 + w (k5 + w k7)), w = u^2, the odd
   // Taylor series of c tanh(u / c) through u^7, used for |u| <= c / 5.
   if (a->softcap > 0.f) {

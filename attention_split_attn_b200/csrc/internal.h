@@ -170,6 +170,14 @@ struct PrefillPlan {
   int32_t out_vec;          // output rows may be written with 16-byte stores
   int32_t mask_vec;         // mask rows may be read with 16-byte loads
   int* status;
+  // Split units: CTAs [0, n_full) are whole units; the next n_split units
+  // run as k_split parts each (CTA n_full + u * k_split + part) whose
+  // (m, l, O) go to part_o / part_ml and are folded by the last part to finish
+  // (split_cnt: one counter per split unit, zeroed by the classifier).
+  int64_t n_full, n_split;
+  int32_t k_split;
+  int* split_cnt;
+  float *part_o, *part_ml;
   uint64_t wait_ns;         // bound of every barrier wait (a timeout records ATTN_ERR_DEVICE_TIMEOUT)
   int32_t test_stall;       // 1: the softmax warps first wait on a barrier nothing arrives at
 };
@@ -194,6 +202,12 @@ struct CombinePlan {
   int use_pdl;
 };
 cudaError_t launch_combine(const CombinePlan& p, cudaStream_t stream);
+
+// ---- masked route of selected-key attention ------------------------------------------
+// Row r of the F32 mask [n_rows][mask_sr]: -inf, 0 at the valid entries of
+// row r's selection list (mask 16-byte aligned, mask_sr a multiple of 4).
+cudaError_t launch_sel_mask(const int32_t* sel, int64_t sel_sr, int32_t n_sel, int32_t n_rows, int32_t n_cells,
+                            float* mask, int64_t mask_sr, cudaStream_t stream);
 
 // ---- draft-tree rows ------------------------------------------------------------
 cudaError_t launch_tree_mask(const int32_t* parent, int32_t n_rows, int32_t prefix_cells, int32_t n_cells,

@@ -253,6 +253,8 @@ __global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPl
   __shared__ int4 rows_sh[kPfRows];
   __shared__ float wmax[kClsThreads / 32];
   const int64_t b = blockIdx.x;
+  if (b == 0)   // the row counters of split units start at zero in every call
+    for (int64_t i = threadIdx.x; i < p.n_split * 2 * kPfRows; i += kClsThreads) p.split_cnt[i] = 0;
   const int64_t n_cls = (int64_t)p.n_rt * p.n_kt;
   if (b < n_cls) {
     pf_classify_tile(p, b, rows_sh);
@@ -398,12 +400,16 @@ struct PfTiles {
   const uint8_t* cls;    // this row tile's class row [n_kt]
   const uint8_t* vbad;   // [n_kt][Hkv]
   int n_kt, Hkv, g;
+  int hi, lo;            // this CTA's tiles: kt in (lo, hi], not skipped (a part of a split unit)
   __device__ __forceinline__ int below(int kt) const {
     while (kt >= 0 && (cls[kt] & 3) == kTileSkip) --kt;
     return kt;
   }
-  __device__ __forceinline__ int first() const { return below(n_kt - 1); }
-  __device__ __forceinline__ int next(int kt) const { return below(kt - 1); }
+  __device__ __forceinline__ int first() const { return hi; }
+  __device__ __forceinline__ int next(int kt) const {
+    const int n = below(kt - 1);
+    return n > lo ? n : -1;
+  }
   // Full, Mixed or Bits; MixedBadV for a non-full tile whose V (this KV head)
   // holds a non-finite value (P V then runs on the CUDA cores).
   __device__ __forceinline__ int code(int kt) const {
@@ -781,10 +787,91 @@ __device__ __forceinline__ void pf_pv_cuda_cores(const uint32_t* pk, const uint3
   tmem_wait_st();
 }
 
+// A CTA's share of a split unit: part `part` of nparts; su = the unit's index
+// among the split units (negative for a whole unit).
+struct PfSplit {
+  int nparts, part;
+  int64_t su;
+};
+
+// The end of a part of a split unit, for one thread's row (kept out of line:
+// it runs once per CTA and would otherwise crowd the softmax loop's
+// registers; every lane of the warp calls it): store this row's (m, l, O),
+// and let the last part to finish (one counter per row) fold all parts in
+// part order with the sink.  Stores before the counter, the counter before
+// the loads.
+template <int D>
+__device__ __noinline__ void pf_split_epilogue(const PrefillPlan& p, const PfSplit& split, uint32_t tO, bool has_o,
+                                               float m, float l, bool rvalid, int r, int h, int slot, int row_t,
+                                               bool out_vec) {
+  constexpr int HPC = PfLayout<D>::HPC;
+  auto rec = [&](int prt) { return ((split.su * split.nparts + prt) * HPC + slot) * kPfRows + row_t; };
+  float* o = p.part_o + rec(split.part) * D;
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t ou[32];
+    if (has_o) {   // every lane of the warp reads tensor memory (.sync.aligned)
+      tmem_ld32(tO + ch * 32, ou);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ou[e] = 0u;
+    }
+    if (rvalid) {
+      float4* dst = reinterpret_cast<float4*>(o + ch * 32);
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4)
+        dst[k4] = make_float4(__uint_as_float(ou[4 * k4]), __uint_as_float(ou[4 * k4 + 1]),
+                              __uint_as_float(ou[4 * k4 + 2]), __uint_as_float(ou[4 * k4 + 3]));
+    }
+  }
+  if (!rvalid) return;
+  p.part_ml[rec(split.part) * 2] = m;
+  p.part_ml[rec(split.part) * 2 + 1] = l;
+  __threadfence();
+  int* cnt = p.split_cnt + (split.su * 2 + slot) * kPfRows + row_t;
+  if (atomicAdd(cnt, 1) != split.nparts - 1) return;   // not the last part
+  *cnt = 0;                                              // ready for the next call
+  __threadfence();
+  const float sigma = p.lg.sinks ? __ldg(p.lg.sinks + h) : neg_inf();
+  float Mf = sigma;
+  for (int q = 0; q < split.nparts; ++q) Mf = fmax_nan(Mf, __ldcg(p.part_ml + rec(q) * 2));
+  const bool is_nan = isnan(Mf), is_zero = (Mf == neg_inf());
+  // weight of part q's O: e^(m_q - M) (0 for an empty part)
+  auto weight = [&](int q) {
+    return (is_nan || is_zero) ? 0.f : ex2((__ldcg(p.part_ml + rec(q) * 2) - Mf) * kLog2e);
+  };
+  float Lf = is_nan || is_zero ? 1.f : ex2((sigma - Mf) * kLog2e);
+  for (int q = 0; q < split.nparts; ++q) Lf = fmaf(__ldcg(p.part_ml + rec(q) * 2 + 1), weight(q), Lf);
+  const float inv = 1.f / Lf;
+  const int64_t ob = (int64_t)r * p.out.sr + (int64_t)h * p.out.sh;
+#pragma unroll 1
+  for (int ch = 0; ch < D / 32; ++ch) {
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+    for (int q = 0; q < split.nparts; ++q) {
+      const float wgt = weight(q);
+      const float4* src = reinterpret_cast<const float4*>(p.part_o + rec(q) * D + ch * 32);
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        const float4 x = __ldcg(src + k4);
+        v[4 * k4] = fmaf(x.x, wgt, v[4 * k4]);
+        v[4 * k4 + 1] = fmaf(x.y, wgt, v[4 * k4 + 1]);
+        v[4 * k4 + 2] = fmaf(x.z, wgt, v[4 * k4 + 2]);
+        v[4 * k4 + 3] = fmaf(x.w, wgt, v[4 * k4 + 3]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = is_nan ? qnan() : (is_zero ? 0.f : v[e] * inv);
+    pf_store32(p.out, ob + ch * 32, v, out_vec);
+  }
+}
+
 template <typename KT, int D>
 __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& tiles, unsigned char* sm,
                                            const PfBars& B, volatile int* abort_flag, uint32_t tmem, int rt,
-                                           int h, int slot, int quarter, int lane) {
+                                           int h, int slot, int quarter, int lane, const PfSplit& split) {
   const bool out_vec = p.out_vec != 0, mask_vec = p.mask_vec != 0;
   using L = PfLayout<D>;
   uint64_t* s_full = B.s_full;
@@ -1028,6 +1115,10 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p, abort_flag)) return;
     tc_fence_after();
   }
+  if (split.nparts > 1) {
+    pf_split_epilogue<D>(p, split, tO, j > 0, m, l, rvalid, r, h, slot, row_t, out_vec);
+    return;
+  }
   // Fold with the sink (an extra logit with no value vector) and normalise.
   const float sigma = p.lg.sinks ? __ldg(p.lg.sinks + h) : neg_inf();
   const float Mf = fmax_nan(m, sigma);
@@ -1075,10 +1166,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // work unit (row tile, KV head, q head pair) and, for a split unit, the part
+  int64_t unit = blockIdx.x;
+  int part = 0, nparts = 1;
+  if (unit >= p.n_full) {
+    const int64_t q = unit - p.n_full;
+    unit = p.n_full + q / p.k_split;
+    part = (int)(q % p.k_split);
+    nparts = p.k_split;
+  }
   const int per_rt = p.Hkv * p.n_pairs;
-  const int rt = p.n_rt - 1 - (int)(blockIdx.x / per_rt);
-  const int g = (int)(blockIdx.x % per_rt) / p.n_pairs;
-  const int pair = (int)(blockIdx.x % per_rt) % p.n_pairs;
+  const int rt = p.n_rt - 1 - (int)(unit / per_rt);
+  const int g = (int)(unit % per_rt) / p.n_pairs;
+  const int pair = (int)(unit % per_rt) % p.n_pairs;
   const int h0 = g * p.G + L::HPC * pair;
   const int n_slots = min(L::HPC, p.G - L::HPC * pair);
 
@@ -1103,14 +1203,42 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
   pdl_wait_prior_grid();   // tile classes from the classifier
 
-  const PfTiles tiles{p.cls + (int64_t)rt * p.n_kt, p.vbad, p.n_kt, p.Hkv, g};
+  PfTiles tiles{p.cls + (int64_t)rt * p.n_kt, p.vbad, p.n_kt, p.Hkv, g, -1, -1};
+  {
+    // This CTA's tiles in walk order (nearest first): all of the row tile's
+    // non-skipped tiles, or part `part` of nparts equal runs of them.  Every
+    // warp finds the same bounds: lane l looks at tile top - l.
+    const uint8_t* cls = tiles.cls;
+    int cnt = 0;
+    for (int base = 0; base < p.n_kt; base += 32) {
+      const int kt = base + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, kt < p.n_kt && (cls[kt] & 3) != kTileSkip));
+    }
+    const int a = (int)((int64_t)part * cnt / nparts), bnd = (int)((int64_t)(part + 1) * cnt / nparts);
+    int hi = -1, lo = -1, running = 0;
+    for (int top = p.n_kt - 1; top >= 0; top -= 32) {
+      const int kt = top - lane;
+      const bool ns = kt >= 0 && (cls[kt] & 3) != kTileSkip;
+      const uint32_t bal = __ballot_sync(0xffffffffu, ns);
+      const int rank = running + __popc(bal & ((1u << lane) - 1u));
+      const uint32_t at_a = __ballot_sync(0xffffffffu, ns && rank == a);
+      const uint32_t at_b = __ballot_sync(0xffffffffu, ns && rank == bnd);
+      if (at_a) hi = top - (__ffs(at_a) - 1);
+      if (at_b) lo = top - (__ffs(at_b) - 1);
+      running += __popc(bal);
+    }
+    if (a >= bnd) hi = -1;   // an empty part (fewer tiles than parts)
+    tiles.hi = hi;
+    tiles.lo = lo;
+  }
+  const PfSplit split{nparts, part, unit - p.n_full};
 
   if (warp >= 4) {
     // ---- softmax warpgroups ----
     setmaxnreg_inc<L::HIGH_REGS>();
     const int slot = (warp >> 2) - 1;
     if (slot < n_slots)
-      pf_softmax<KT, D>(p, tiles, sm, B, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane);
+      pf_softmax<KT, D>(p, tiles, sm, B, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane, split);
   } else {
   setmaxnreg_dec<L::LOW_REGS>();
   if (warp == 0) {
@@ -1236,10 +1364,14 @@ cudaError_t launch_prefill_t(const PrefillPlan& p, const CUtensorMap& tmQ, const
   if (n_cls + n_scan > 0) {
     prefill_classify_kernel<<<(unsigned)(n_cls + n_scan), kClsThreads, 0, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else if (p.n_split > 0) {
+    // no classifier runs (no cells): zero the split units' row counters here
+    if ((e = cudaMemsetAsync(p.split_cnt, 0, (size_t)p.n_split * 2 * kPfRows * sizeof(int), stream)) != cudaSuccess)
+      return e;
   }
   if (after_classify) cudaEventRecord(after_classify, stream);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((int64_t)p.n_rt * p.Hkv * p.n_pairs));
+  cfg.gridDim = dim3((unsigned)(p.n_full + p.n_split * p.k_split));
   cfg.blockDim = dim3(L::THREADS);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = stream;

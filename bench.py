@@ -395,6 +395,12 @@ def selected_bytes(p) -> int:
     return kv + p.q.numel() * p.q.element_size() + sel.size * 4 + o
 
 
+def _selected_pairs(p) -> int:
+    """Distinct valid selected (row, cell) pairs."""
+    sel = p.sel.numpy()
+    return sum(len(np.unique(row[(row >= 0) & (row < p.n_cells)])) for row in sel)
+
+
 def prefill_flops(p) -> int:
     """4 D flops (QK^T and PV) per visible (row, cell, q head); visibility is
     carried by the mask in the causal prefill workload."""
@@ -470,7 +476,32 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
     if with_cpu:
         parts["selected"]["cpu_baseline"] = _part_baseline(p, list(range(0, 2048, 128)), selected_bytes, "GB/s",
                                                            1e9, "16 of the 2048 rows (every 128th)")
-    del q, k, v, out, sel, sa, ws, kw
+    del sa, ws
+
+    # the masked per-cell route on the same workload (strix-llama.cpp PR #115,
+    # "Measurements"): a dense F32 mask [2048 x 32768] from the lists, then the
+    # tensor-core prefill kernel; same result, same effective-bytes metric
+    ma = A.make_selected_args(q, k, v, out, sel, **kw)
+    mws = torch.empty(max(A.selected_masked_workspace_size(ma), 256), dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        A.attn_selected_masked_args(ma, ws=mws, stream=stream)
+    nm = max(3, min(args.steps, 5))
+    whole_m, main_m = _time_calls(lambda e: A.attn_selected_masked_timed_args(ma, mws, e, stream=stream), nm,
+                                  flush, stream)
+    sflops = 4 * p.head_dim * p.n_head_q * _selected_pairs(p)
+    parts["selected_masked"] = {
+        "workload": "selected_prefill through the masked per-cell route: F32 mask 2048 x 32768 from the lists, "
+                    "then the dense tensor-core pass (tile classifier skips tiles no row selected)",
+        "value": nbytes / (whole_m * 1e-3) / 1e9, "unit": "GB/s (effective: gathered K/V bytes, as selected)",
+        "ms_per_call": whole_m, "vs_selected_kernel": whole_m / whole, "calls": nm,
+        "gpu_launches": 3 * nm,   # mask builder + tile classifier + tensor-core kernel
+        "roofline": {"bound": "tensor", "achieved": sflops / (main_m * 1e-3) / 1e12, "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": sflops / (main_m * 1e-3) / 1e12 / tc_peak, "traffic": None,
+                     "kernel": "sel_mask_kernel + prefill_classify_kernel + prefill_kernel<f16, 256>",
+                     "kernel_ms": main_m, "algorithmic_flops": sflops,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS); flops of the selected pairs only"},
+    }
+    del q, k, v, out, sel, ma, mws, kw
 
     # causal prefill: 2048 rows over 14048 cells, Hq 64 / Hkv 8, D 128, bf16
     p = W.causal_prefill()

@@ -132,7 +132,7 @@ typedef enum {
     ATTN_ERR_DEVICE_TIMEOUT = -5   /* a kernel gave up waiting on a barrier          */
 } attn_status;
 
-enum { ATTN_OP_DECODE = 0, ATTN_OP_SELECTED = 1, ATTN_OP_PREFILL = 2 };
+enum { ATTN_OP_DECODE = 0, ATTN_OP_SELECTED = 1, ATTN_OP_PREFILL = 2, ATTN_OP_SELECTED_MASKED = 3 };
 
 /* Shared argument block (see the file comment for meaning and layout). */
 typedef struct {
@@ -190,7 +190,7 @@ typedef struct {
 } attn_selected_args;
 
 /* Workspace bytes the op needs for these arguments (0 is possible).  n_sel is
- * used by ATTN_OP_SELECTED only.  Returns 0 also for invalid arguments; call
+ * used by ATTN_OP_SELECTED and ATTN_OP_SELECTED_MASKED only.  Returns 0 also for invalid arguments; call
  * attn_supports() to tell the two apart.                                     */
 size_t attn_workspace_size(const attn_args *args, int32_t op, int32_t n_sel);
 
@@ -217,6 +217,25 @@ int32_t attn_selected_timed(const attn_selected_args *args, void *ws, size_t ws_
                             void *const events[3]);
 int32_t attn_prefill_timed(const attn_args *args, void *ws, size_t ws_bytes, void *stream,
                            void *const events[3]);
+
+/* The masked per-cell route of selected-key attention (strix-llama.cpp PR
+ * #115, "Measurements": the route a backend without the selected-key kernels
+ * takes, a dense per-cell mask over the cache).  Same arguments and result as
+ * attn_selected: it writes each row's F32 mask [n_cells] into the workspace
+ * (-inf, 0 at every valid listed cell) and runs the attn_prefill tensor-core
+ * kernel on it, whose tile classifier skips the tiles no row of a row tile
+ * selected.  Takes what that kernel takes (Q in the K/V dtype, F16/BF16,
+ * head_dim 64, 128 or 256); cell_pos/row_pos serve ALiBi as in attn_selected
+ * (NULL: cell c at c, every row at n_cells - 1).  sel_sorted_out /
+ * sel_count_out are not written.  Workspace: attn_workspace_size(base,
+ * ATTN_OP_SELECTED_MASKED, n_sel) -- the mask (n_rows x n_cells floats, rows
+ * padded to 4) first, then the dense pass's workspace; it grows with the
+ * cache, which is the point of the selected-key kernel.  The timed form
+ * records events[0] before the mask kernel and events[1], events[2] as
+ * attn_prefill_timed does.                                                  */
+int32_t attn_selected_masked(const attn_selected_args *args, void *ws, size_t ws_bytes, void *stream);
+int32_t attn_selected_masked_timed(const attn_selected_args *args, void *ws, size_t ws_bytes, void *stream,
+                                   void *const events[3]);
 
 /* attn_decode for callers that cannot allocate device memory (a real-time
  * loop that must not block in an allocator, a plugin with no memory pool of
