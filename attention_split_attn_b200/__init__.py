@@ -34,6 +34,7 @@ _DTYPE = {torch.float32: ATTN_F32, torch.float16: ATTN_F16, torch.bfloat16: ATTN
 EXPORTS = ("attn_workspace_size", "attn_supports", "attn_decode", "attn_selected",
            "attn_prefill", "attn_decode_timed", "attn_selected_timed", "attn_prefill_timed",
            "attn_decode_noalloc", "attn_tree_mask", "attn_selected_masked", "attn_selected_masked_timed",
+           "attn_decode_append", "attn_decode_cluster",
            "attn_check_device_status",
            "attn_strerror", "attn_last_error", "attn_abi_version")
 
@@ -115,6 +116,12 @@ def load_library():
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int32
                 fn.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            lib.attn_decode_cluster.restype = ctypes.c_int32
+            lib.attn_decode_cluster.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
+            lib.attn_decode_append.restype = ctypes.c_int32
+            lib.attn_decode_append.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t,
+                                               ctypes.c_void_p]
             lib.attn_selected_masked_timed.restype = ctypes.c_int32
             lib.attn_selected_masked_timed.argtypes = [ctypes.POINTER(AttnSelectedArgs), ctypes.c_void_p,
                                                        ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p * 3]
@@ -230,6 +237,34 @@ def attn_decode_args(args: AttnArgs, ws: Optional[torch.Tensor] = None, stream=N
                          0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
     _raise_if(st, "attn_decode")
     return ws
+
+
+def attn_decode_append_args(args: AttnArgs, k_new: torch.Tensor, v_new: torch.Tensor,
+                            ws: Optional[torch.Tensor] = None, stream=None):
+    """attn_decode with the step's cache append fused in (see include/attn.h):
+    k_new / v_new [rows, n_head_kv, head_dim] in the cache dtype go to cell
+    row_end[r] - 1 of the cache the AttnArgs points at."""
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if t.dim() != 3 or t.stride(2) != 1 or t.dtype not in _DTYPE:
+            raise ValueError(f"{name} must be [rows, n_head_kv, head_dim] with the head dimension contiguous")
+    if k_new.stride() != v_new.stride():
+        raise ValueError("k_new and v_new must share strides")
+    lib = load_library()
+    need = workspace_size(args, OP_DECODE)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = _workspace(need, dev, ws)
+    st = lib.attn_decode_append(ctypes.byref(args), k_new.data_ptr(), v_new.data_ptr(), k_new.stride(0),
+                                k_new.stride(1), None if ws is None else ws.data_ptr(),
+                                0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
+    _raise_if(st, "attn_decode_append")
+    return ws
+
+
+def attn_decode_cluster_args(args: AttnArgs, stream=None):
+    """attn_decode through one 8-CTA cluster per (row, KV head), partials folded
+    over distributed shared memory (no workspace; see include/attn.h)."""
+    lib = load_library()
+    _raise_if(lib.attn_decode_cluster(ctypes.byref(args), _stream_handle(stream)), "attn_decode_cluster")
 
 
 def attn_decode_timed_args(args: AttnArgs, ws: Optional[torch.Tensor], events, stream=None):

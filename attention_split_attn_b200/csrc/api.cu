@@ -618,8 +618,84 @@ int32_t attn_decode(const attn_args* a, void* ws, size_t ws_bytes, void* stream)
   return attn_decode_timed(a, ws, ws_bytes, stream, nullptr);
 }
 
+// New K/V rows of attn_decode_append.
+struct AppendSpec {
+  const void *k_new, *v_new;
+  int64_t sr, sh;
+};
+
+int32_t decode_run(const attn_args* a, void* ws, size_t ws_bytes, void* stream, void* const events[3],
+                   const AppendSpec* app);
+
 int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* stream,
                           void* const events[3]) {
+  return decode_run(a, ws, ws_bytes, stream, events, nullptr);
+}
+
+int32_t attn_decode_append(const attn_args* a, const void* k_new, const void* v_new, int64_t new_stride_row,
+                           int64_t new_stride_head, void* ws, size_t ws_bytes, void* stream) {
+  int32_t st = check_decode(a);
+  if (st != ATTN_OK) return st;
+  if (a->n_rows == 0) return ATTN_OK;
+  if (!k_new || !v_new) return fail(ATTN_ERR_INVALID_ARG, "append: k_new or v_new is NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || (a->n_rows > 1 && new_stride_row % 8) ||
+      (a->n_head_kv > 1 && new_stride_head % 8))
+    return fail(ATTN_ERR_UNSUPPORTED, "append: new rows must be 16-byte aligned with strides that are multiples of 8");
+  if (new_stride_head < a->head_dim || (a->n_rows > 1 && new_stride_row < (int64_t)a->n_head_kv * new_stride_head))
+    return fail(ATTN_ERR_INVALID_ARG, "append: new row strides overlap");
+  if (!a->row_end && a->n_rows > 1)
+    return fail(ATTN_ERR_INVALID_ARG, "append: with several rows, row_end must say where each row's token goes");
+  if (unified_route(a) || a->n_slices != 0 || !decode_uses_mma(a->kv_type, a->q_type, a->q, a->q_stride_row,
+                                                                 a->q_stride_head))
+    return fail(ATTN_ERR_UNSUPPORTED,
+                "append: runs on the balanced tensor-core kernel (16-bit cache, Q in its dtype, n_slices 0, "
+                "no per-cell sequence ids)");
+  const AppendSpec app{k_new, v_new, new_stride_row, new_stride_head};
+  return decode_run(a, ws, ws_bytes, stream, nullptr, &app);
+}
+
+int32_t attn_decode_cluster(const attn_args* a, void* stream) {
+  int32_t st = check_decode(a);
+  if (st != ATTN_OK) return st;
+  const int G = a->n_head_q / a->n_head_kv;
+  if (unified_route(a) || a->n_slices != 0 || (a->head_dim != 64 && a->head_dim != 128) ||
+      !decode_uses_mma(a->kv_type, a->q_type, a->q, a->q_stride_row, a->q_stride_head))
+    return fail(ATTN_ERR_UNSUPPORTED,
+                "cluster decode: a 16-bit cache with Q in its dtype, head_dim 64 or 128, n_slices 0, no per-cell "
+                "sequence ids");
+  if (a->n_rows == 0) return ATTN_OK;
+  if ((int64_t)a->n_rows * a->n_head_kv * 8 > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+  DeviceInfo* di = nullptr;
+  if ((st = device_info(&di)) != ATTN_OK) return st;
+  CUtensorMap tmK, tmV;
+  memset(&tmK, 0, sizeof(tmK));
+  memset(&tmV, 0, sizeof(tmV));
+  if (a->n_cells > 0) {
+    if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                          a->kv_stride_head, 16, 64, true)) != ATTN_OK)
+      return st;
+    if ((st = make_kv_map(&tmV, a->v, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
+                          a->kv_stride_head, 16, 64, true)) != ATTN_OK)
+      return st;
+  }
+  DecodePlan p{};
+  p.R = a->n_rows; p.Hq = a->n_head_q; p.Hkv = a->n_head_kv; p.G = G;
+  p.D = a->head_dim; p.N = a->n_cells;
+  p.q = QSpec{a->q, a->q_type, a->q_stride_row, a->q_stride_head};
+  p.out = OutSpec{a->out, a->out_type, a->o_stride_row, a->o_stride_head};
+  p.f = RowFilter{a->row_begin, a->row_end, a->cell_seq, a->row_seq, a->cell_pos, a->row_pos,
+                  a->causal, a->mask, a->mask_stride_row};
+  p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
+  p.kv_type = a->kv_type;
+  p.mma = 1;
+  p.status = di->status;
+  const cudaError_t e = launch_decode_cluster(p, tmK, tmV, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cluster decode launch: %s", cudaGetErrorString(e));
+  return ATTN_OK;
+}
+
+int32_t decode_run(const attn_args* a, void* ws, size_t ws_bytes, void* stream, void* const events[3],
+                   const AppendSpec* app) {
   int32_t st = check_decode(a);
   if (st != ATTN_OK) return st;
   if (a->n_rows == 0) return ATTN_OK;
@@ -664,6 +740,11 @@ int32_t attn_decode_timed(const attn_args* a, void* ws, size_t ws_bytes, void* s
   p.S = sh.S; p.C = sh.C; p.grid_order = a->grid_order;
   p.hpw = sh.hpw; p.hg = sh.hg; p.kv_type = a->kv_type; p.mma = mma ? 1 : 0;
   p.k_scale = a->k_scale; p.v_scale = a->v_scale; p.scale_sc = a->scale_stride_cell;
+  if (app) {
+    p.k_new = app->k_new; p.v_new = app->v_new; p.new_sr = app->sr; p.new_sh = app->sh;
+    p.k_out = const_cast<void*>(a->k); p.v_out = const_cast<void*>(a->v);
+    p.kv_sc = a->kv_stride_cell; p.kv_sh = a->kv_stride_head;
+  }
   p.status = di->status;
   const DecodeWs wl = decode_ws_layout(a, sh);
   char* wsb = static_cast<char*>(ws);

@@ -159,6 +159,35 @@ __device__ __forceinline__ void cursor_next(const DecodePlan& p, const int64_t* 
   } while (c.nt == 0 && c.r + 1 < p.R);
 }
 
+// Fused append: when this tile holds the append cell of its (row, KV head)
+// (cell row_end - 1), write the row's new K and V into the cache and over the
+// staged copy of that cell (the TMA may have read the cell before or after
+// the cache write), so the attention of this launch already sees them.  Each
+// (row, KV head, tile) belongs to exactly one warp, so each new row is
+// written once.  16-byte chunks, one per lane per pass; the staged rows are
+// 128-byte swizzled (chunk k of cell row i at chunk k ^ (i & 7)).
+template <int D>
+__device__ __forceinline__ void append_patch(const DecodePlan& p, const Cursor& c, unsigned char* stage, int lane) {
+  const int t0 = c.begin + (int)(c.j * kWarpTile);
+  const int a = c.raw_e - 1;   // the append cell (inside [begin, end) whenever the row has cells)
+  if (a < t0 || a >= t0 + kWarpTile || a < c.begin || a >= c.end) return;
+  const int row = a - t0;
+  constexpr int CH = D / 8;    // 16-byte chunks of one cell row of one head
+  const int64_t src = (int64_t)c.r * p.new_sr + (int64_t)c.g * p.new_sh;
+  const int64_t dst = (int64_t)a * p.kv_sc + (int64_t)c.g * p.kv_sh;
+  for (int i = lane; i < 2 * CH; i += 32) {
+    const bool is_v = i >= CH;
+    const int ch = is_v ? i - CH : i;
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(is_v ? p.v_new : p.k_new) + src) + ch);
+    reinterpret_cast<uint4*>(static_cast<uint16_t*>(is_v ? p.v_out : p.k_out) + dst)[ch] = w;
+    const int sub = ch >> 3, k = ch & 7;
+    const uint32_t off = (is_v ? (uint32_t)(kWarpTile * D * 2) : 0u) + (uint32_t)sub * (kWarpTile * 128) +
+                         (uint32_t)row * 128u + ((uint32_t)(k ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4*>(stage + off) = w;
+  }
+  __syncwarp();
+}
+
 template <typename KT, int D, int NH>
 __global__ void __launch_bounds__(32)
 decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -274,6 +303,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       break;
     }
     unsigned char* stage = smem + stg * Ring::STAGE;
+    if (Tr::ES == 2 && p.k_new) append_patch<D>(p, c, stage, lane);
     st.load_tile(stage);
     auto refill = [&]() {
       __syncwarp();
@@ -373,7 +403,211 @@ int stream_blocks_per_sm() {
   return n;
 }
 
+// ---------------------------------------------------------------------------
+// cluster decode: one thread-block cluster per (row, KV head)
+// ---------------------------------------------------------------------------
+// A latency variant for few, long rows (TensorFold PR #985, change list: a
+// cluster of CTAs shares a head over distributed shared memory).  The row's
+// 16-cell tiles of one KV head are cut into kClWarps * kClCtas equal runs;
+// each warp of each CTA of the cluster folds its run with the tensor-core
+// tile step (its own TMA ring, as in the stream kernel) and leaves its
+// partial (m, l, O) in its CTA's shared memory; after a cluster barrier CTA
+// rank 0 reads all partials over distributed shared memory and folds them in
+// (rank, warp) order with the sink -- no workspace, no combine launch.  Both
+// cluster barriers are reached on every path (a warp whose bounded wait runs
+// out poisons its partial and drains its copies), so no CTA waits forever.
+constexpr int kClCtas = 8;    // CTAs per cluster (the portable maximum)
+constexpr int kClWarps = 8;   // warps per CTA
+
+template <int D, int NH>
+struct ClusterSmem {
+  using Ring = StreamRing<D, 2>;
+  static constexpr int RING = Ring::NS * Ring::STAGE;           // one warp's stages
+  static constexpr int BARS = kClWarps * RING;                  // [kClWarps][NS] mbarriers
+  static constexpr int PART_O = BARS + kClWarps * Ring::NS * 8; // [kClWarps][NH][D] floats
+  static constexpr int PART_ML = PART_O + kClWarps * NH * D * 4;  // [kClWarps][NH][2]
+  static constexpr int TOTAL = PART_ML + kClWarps * NH * 2 * 4 + 1024;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster(const void* local, uint32_t rank) {
+  uint32_t a = smem_u32(local), ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+template <typename KT, int D, int NH>
+__global__ void __launch_bounds__(32 * kClWarps)
+decode_cluster_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const DecodePlan p) {
+  using Sm = ClusterSmem<D, NH>;
+  using Ring = typename Sm::Ring;
+  constexpr int NS = Ring::NS;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = align1024(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int unit = blockIdx.x / kClCtas;
+  const int r = unit / p.Hkv, g = unit % p.Hkv;
+  unsigned char* ring = smem + warp * Sm::RING;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::BARS) + warp * NS;
+  float* part_o = reinterpret_cast<float*>(smem + Sm::PART_O);
+  float* part_ml = reinterpret_cast<float*>(smem + Sm::PART_ML);
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // this warp's run of the (row, KV head)'s tiles
+  Cursor c;
+  c.r = r;
+  c.g = g;
+  c.raw_b = p.f.row_begin ? __ldg(p.f.row_begin + r) : 0;
+  c.raw_e = p.f.row_end ? __ldg(p.f.row_end + r) : p.N;
+  c.begin = max(c.raw_b, 0);
+  c.end = max(min(c.raw_e, p.N), c.begin);
+  const int64_t nt = (c.end - c.begin + kWarpTile - 1) / kWarpTile;
+  const int share = (int)rank * kClWarps + warp, n_share = kClCtas * kClWarps;
+  const int64_t t0 = nt * share / n_share, t1 = nt * (share + 1) / n_share;
+  const int64_t n = t1 - t0;
+  uint64_t pol = 0;
+  int64_t issued = 0;
+  if (lane == 0) {
+    pol = policy_evict_first();
+    for (; issued < (n < NS ? n : (int64_t)NS); ++issued)
+      issue_stream_tile<D, 2>(ring + issued * Ring::STAGE, &full[issued], &tmK, &tmV, g,
+                              c.begin + (int)((t0 + issued) * kWarpTile), pol);
+  }
+  const bool has_filter = (p.f.cell_seq && p.f.row_seq) || p.f.causal || p.f.mask;
+  RowCtx rc;
+  rc.begin = c.begin;
+  rc.end = c.end;
+  rc.pos_base = c.raw_b;
+  rc.s_begin = c.begin;
+  rc.s_end = c.end;
+  rc.row_seq = p.f.row_seq ? __ldg(p.f.row_seq + r) : 0;
+  rc.row_pos = p.f.row_pos ? (int64_t)__ldg(p.f.row_pos + r) : (int64_t)c.raw_e - c.raw_b - 1;
+  WarpTileState<KT, D, NH> st;
+  st.reset();
+  st.init_offsets(lane);
+  st.load_q(p, r, g * p.G, lane);
+  bool aborted = false;
+  int64_t k = 0;
+  for (; k < n; ++k) {
+    const int stg = (int)(k % NS);
+    if (!mbar_wait_bounded(&full[stg], (uint32_t)((k / NS) & 1), p.status)) {
+      aborted = true;
+      break;
+    }
+    unsigned char* stage = ring + stg * Ring::STAGE;
+    st.load_tile(stage);
+    auto refill = [&]() {
+      __syncwarp();
+      if (lane == 0 && issued < n) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_stream_tile<D, 2>(stage, &full[stg], &tmK, &tmV, g, c.begin + (int)((t0 + issued) * kWarpTile), pol);
+        ++issued;
+      }
+    };
+    if (decltype(st)::kEarlyRelease) refill();
+    st.compute(p, rc, r, c.begin + (int)((t0 + k) * kWarpTile), has_filter, lane, stage);
+    if (!decltype(st)::kEarlyRelease) refill();
+  }
+  if (aborted && lane == 0)   // leave no copy in flight
+    for (int64_t kk = k; kk < issued; ++kk) mbar_wait_bounded(&full[kk % NS], (uint32_t)((kk / NS) & 1), nullptr);
+  st.finish_sums();
+  // this warp's partial: [NH][D] and [NH][2] in its slot of the CTA's shared memory
+  st.write_partial(part_o + warp * NH * D, part_ml + warp * NH * 2, 0, NH, lane, aborted);
+  cluster_sync_all();   // every CTA's partials are in place
+  if (rank == 0) {
+    // fold the kClCtas x kClWarps partials in (rank, warp) order with the sink:
+    // thread t takes head t / 32 (t < 32 G), dims lane, lane + 32, ...
+    const int hh = threadIdx.x >> 5;
+    for (int h = hh; h < p.G; h += kClWarps) {
+      const int hq = g * p.G + h;
+      const float sigma = p.lg.sinks ? __ldg(p.lg.sinks + hq) : neg_inf();
+      float M = sigma;
+      for (int q = 0; q < n_share; ++q) {
+        const float mq = ld_cluster(part_ml + ((q % kClWarps) * NH + h) * 2, (uint32_t)(q / kClWarps));
+        M = fmax_nan(M, mq);
+      }
+      const bool is_nan = isnan(M), is_zero = (M == neg_inf());
+      float L = (is_nan || is_zero) ? 1.f : ex2((sigma - M) * kLog2e);
+      for (int q = 0; q < n_share; ++q) {
+        const uint32_t rk = (uint32_t)(q / kClWarps);
+        const float* ml = part_ml + ((q % kClWarps) * NH + h) * 2;
+        const float mq = ld_cluster(ml, rk);
+        const float wq = (is_nan || is_zero) ? 0.f : ex2((mq - M) * kLog2e);
+        L = fmaf(ld_cluster(ml + 1, rk), wq, L);
+      }
+      const int64_t ob = (int64_t)r * p.out.sr + (int64_t)hq * p.out.sh;
+      for (int d = lane; d < D; d += 32) {
+        float o = 0.f;
+        for (int q = 0; q < n_share; ++q) {
+          const uint32_t rk = (uint32_t)(q / kClWarps);
+          const float mq = ld_cluster(part_ml + ((q % kClWarps) * NH + h) * 2, rk);
+          const float wq = (is_nan || is_zero) ? 0.f : ex2((mq - M) * kLog2e);
+          o = fmaf(ld_cluster(part_o + ((q % kClWarps) * NH + h) * D + d, rk), wq, o);
+        }
+        const float v = is_nan ? qnan() : is_zero ? 0.f : o / L;
+        store_from_float(p.out.out, ob + d, p.out.type, v);
+      }
+    }
+  }
+  cluster_sync_all();   // no CTA leaves while rank 0 may still read its shared memory
+}
+
+template <typename KT, int D, int NH>
+cudaError_t launch_cluster_t(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                             cudaStream_t stream) {
+  using Sm = ClusterSmem<D, NH>;
+  auto kern = decode_cluster_kernel<KT, D, NH>;
+  static std::atomic<unsigned long long> smem_set{0ull};
+  cudaError_t e = set_smem_limit_once(smem_set, kern, Sm::TOTAL);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((int64_t)p.R * p.Hkv * kClCtas));
+  cfg.blockDim = dim3(32 * kClWarps);
+  cfg.dynamicSmemBytes = Sm::TOTAL;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kClCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmK, tmV, p);
+}
+
 }  // namespace
+
+cudaError_t launch_decode_cluster(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                  cudaStream_t stream) {
+  const bool bf = p.kv_type == ATTN_BF16, h16 = p.G > 8;
+  switch (p.D) {
+    case 64:
+      return bf ? (h16 ? launch_cluster_t<__nv_bfloat16, 64, 16>(p, tmK, tmV, stream)
+                       : launch_cluster_t<__nv_bfloat16, 64, 8>(p, tmK, tmV, stream))
+                : (h16 ? launch_cluster_t<__half, 64, 16>(p, tmK, tmV, stream)
+                       : launch_cluster_t<__half, 64, 8>(p, tmK, tmV, stream));
+    default:
+      return bf ? (h16 ? launch_cluster_t<__nv_bfloat16, 128, 16>(p, tmK, tmV, stream)
+                       : launch_cluster_t<__nv_bfloat16, 128, 8>(p, tmK, tmV, stream))
+                : (h16 ? launch_cluster_t<__half, 128, 16>(p, tmK, tmV, stream)
+                       : launch_cluster_t<__half, 128, 8>(p, tmK, tmV, stream));
+  }
+}
 
 int decode_stream_warps(int kv_type, int D, int G, int sms) {
   int per_sm;

@@ -68,6 +68,13 @@ struct DecodePlan {
   // e4m3 / int8 caches: per (cell, KV head) scales at c * scale_sc + g
   const float *k_scale, *v_scale;
   int64_t scale_sc;
+  // fused append (attn_decode_append; balanced 16-bit kernel): row r's new K/V
+  // rows [Hkv][D] at k_new + r * new_sr + g * new_sh go to cell row_end[r] - 1
+  // of the cache (k_out / v_out: the cache, written)
+  const void *k_new, *v_new;
+  int64_t new_sr, new_sh;
+  void *k_out, *v_out;
+  int64_t kv_sc, kv_sh;
 };
 
 bool decode_uses_mma(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh);
@@ -80,6 +87,11 @@ cudaError_t launch_decode_slices(const DecodePlan& p, const CUtensorMap& tmK, co
 // Balanced persistent scheme: planner kernel, then W single-warp CTAs that
 // each take an equal run of the flattened (row, KV head, 16-cell tile) space.
 int decode_stream_warps(int kv_type, int D, int G, int sms);
+// Cluster decode (attn_decode_cluster): one 8-CTA cluster per (row, KV head),
+// partials folded over distributed shared memory; 16-bit caches, head dim
+// 64 or 128.
+cudaError_t launch_decode_cluster(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                  cudaStream_t stream);
 // One-byte caches (e4m3 / int8) that the balanced tensor-core kernel takes.
 bool decode_stream8_supported(int kv_type, int q_type, const void* q, int64_t q_sr, int64_t q_sh, int D, int G);
 cudaError_t launch_decode_stream(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,

@@ -575,6 +575,47 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
             p, list(range(p.n_rows)), lambda s_: tbytes, "GB/s", 1e9, "all 16 rows")
     del q, k, v, out, ta, ws, kw, tmask
 
+    # one long row (130856 cached keys, the depth of TensorFold PR #2595's
+    # long-context receipt), Hq 32 / Hkv 8, D 128, bf16: attn_decode (balanced
+    # kernel + split_k_reduce), attn_decode_cluster (8-CTA clusters, DSMEM
+    # fold, no workspace) and attn_decode_append (the step's append fused in)
+    p = W.random_problem(1010, R=1, Hq=32, Hkv=8, D=128, N=130857, kv_dtype=torch.bfloat16,
+                         out_dtype=torch.bfloat16, lengths=[130857])
+    (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+    la = A.make_args(q, k, v, out, **kw)
+    ws = torch.empty(max(A.workspace_size(la, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+    kn = torch.randn((1, 8, 128), device=dev).to(torch.bfloat16)
+    vn = torch.randn((1, 8, 128), device=dev).to(torch.bfloat16)
+    lbytes = algorithmic_bytes(p)
+    calls = {
+        "decode": lambda: A.attn_decode_args(la, ws=ws, stream=stream),
+        "cluster": lambda: A.attn_decode_cluster_args(la, stream=stream),
+        "append": lambda: A.attn_decode_append_args(la, kn, vn, ws=ws, stream=stream),
+    }
+    lat = {}
+    for name, fn in calls.items():
+        for _ in range(max(args.warmup, 3)):
+            fn()
+
+        def timed(e, fn=fn):
+            e[0].record(stream)
+            fn()
+            e[1].record(stream)
+            e[2].record(stream)
+        lat[name], _ = _time_calls(timed, n, flush, stream)
+    parts["long_row_decode"] = {
+        "workload": "long_row_decode: 1 row over 130857 cached keys, Hq 32 / Hkv 8, D 128, bf16 KV and out",
+        "value": lbytes / (lat["cluster"] * 1e-3) / 1e9, "unit": "GB/s (attn_decode_cluster; K/V, Q, out)",
+        "ms_per_call": lat["cluster"], "ms_attn_decode": lat["decode"], "ms_attn_decode_append": lat["append"],
+        "GBs_attn_decode": lbytes / (lat["decode"] * 1e-3) / 1e9, "calls": n,
+        "gpu_launches": n * (1 + 2 + 2),   # cluster; decode (stream + combine); append (stream + combine)
+        "roofline": {"bound": "hbm", "achieved": lbytes / (lat["cluster"] * 1e-3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": lbytes / (lat["cluster"] * 1e-3) / 1e9 / hbm_peak, "traffic": None,
+                     "kernel": "decode_cluster_kernel (one launch)", "kernel_ms": lat["cluster"],
+                     "algorithmic_bytes": lbytes, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
+    }
+    del q, k, v, out, la, ws, kw
+
     # quantized GQA decode: the decode batch's shape (16 rows, lengths U[1024,
     # 8192], Hq 32 / Hkv 8, D 128) over an e4m3 cache with one F32 scale per
     # (cell, KV head) for K and for V (TensorFold PR #911).  Bytes: the K and V

@@ -218,6 +218,34 @@ int32_t attn_selected_timed(const attn_selected_args *args, void *ws, size_t ws_
 int32_t attn_prefill_timed(const attn_args *args, void *ws, size_t ws_bytes, void *stream,
                            void *const events[3]);
 
+/* attn_decode with the step's K/V cache append fused into the same launch
+ * (TensorFold PR #985, change list: for a single row the attention launch
+ * also does the cache append).  Row r's new K and V rows (k_new, v_new: DEVICE,
+ * the cache dtype, [n_rows][n_head_kv][head_dim] with the given element
+ * strides, 16-byte aligned) are written into cell row_end[r] - 1 of the cache
+ * (args->k / args->v, written here) and the attention of the call already
+ * sees them: the result and the cache are those of an append followed by
+ * attn_decode, bit for bit.  Runs on the balanced tensor-core kernel: a
+ * 16-bit cache with Q in its dtype, n_slices 0, no per-cell sequence ids;
+ * row_end must be given when n_rows > 1 (NULL with one row: cell n_cells - 1),
+ * and row_end[r] - 1 must lie in [row_begin[r], n_cells).  No row's range may
+ * include another row's append cell (rows of separate sequences).  Workspace
+ * as attn_decode.                                                           */
+int32_t attn_decode_append(const attn_args *args, const void *k_new, const void *v_new, int64_t new_stride_row,
+                           int64_t new_stride_head, void *ws, size_t ws_bytes, void *stream);
+
+/* attn_decode for few, long rows without a workspace: one thread-block
+ * cluster of 8 CTAs per (row, KV head) (TensorFold PR #985, change list: a
+ * cluster of CTAs shares a head over distributed shared memory).  Each of the
+ * cluster's 64 warps folds an equal run of the row's 16-cell tiles on the
+ * tensor cores; CTA rank 0 then reads the 64 partials over distributed shared
+ * memory and folds them in order with the sink -- one launch, no workspace,
+ * no split_k_reduce pass.  Same arguments and result as attn_decode (bit-
+ * identical across runs); takes a 16-bit cache with Q in its dtype, head_dim
+ * 64 or 128, up to 16 q heads per KV head, n_slices 0, no per-cell sequence
+ * ids.  Intended for few rows (n_rows x n_head_kv clusters of 8 CTAs).     */
+int32_t attn_decode_cluster(const attn_args *args, void *stream);
+
 /* The masked per-cell route of selected-key attention (strix-llama.cpp PR
  * #115, "Measurements": the route a backend without the selected-key kernels
  * takes, a dense per-cell mask over the cache).  Same arguments and result as
