@@ -261,7 +261,7 @@ def attn_decode_append_args(args: AttnArgs, k_new: torch.Tensor, v_new: torch.Te
 
 
 def attn_decode_cluster_args(args: AttnArgs, stream=None):
-    """attn_decode through one 8-CTA cluster per (row, KV head), partials folded
+    """attn_decode through one 16-CTA cluster per (row, KV head), partials folded
     over distributed shared memory (no workspace; see include/attn.h)."""
     lib = load_library()
     _raise_if(lib.attn_decode_cluster(ctypes.byref(args), _stream_handle(stream)), "attn_decode_cluster")

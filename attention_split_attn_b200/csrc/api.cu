@@ -664,7 +664,7 @@ int32_t attn_decode_cluster(const attn_args* a, void* stream) {
                 "cluster decode: a 16-bit cache with Q in its dtype, head_dim 64 or 128, n_slices 0, no per-cell "
                 "sequence ids");
   if (a->n_rows == 0) return ATTN_OK;
-  if ((int64_t)a->n_rows * a->n_head_kv * 8 > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+  if ((int64_t)a->n_rows * a->n_head_kv * 16 > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != ATTN_OK) return st;
   CUtensorMap tmK, tmV;

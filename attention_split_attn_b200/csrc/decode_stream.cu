@@ -296,8 +296,17 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
   bool aborted = false;
   int64_t k = 0;
+  if constexpr (Tr::ES == 1) st.prefetch(p, c.g, c.begin + (int)(c.j * kWarpTile), lane);
   for (; k < n; ++k) {
     const int stg = (int)(k % NS);
+    if constexpr (Tr::ES == 1) {
+      st.take_prefetched();
+      if (k + 1 < n) {   // the next tile's per-cell scales, a tile ahead
+        Cursor nc = c;
+        cursor_next(p, row_tiles, nc);
+        st.prefetch(p, nc.g, nc.begin + (int)(nc.j * kWarpTile), lane);
+      }
+    }
     if (!mbar_wait_bounded(&full[stg], (uint32_t)((k / NS) & 1), p.status)) {
       aborted = true;
       break;
@@ -408,7 +417,8 @@ int stream_blocks_per_sm() {
 // ---------------------------------------------------------------------------
 // A latency variant for few, long rows (TensorFold PR #985, change list: a
 // cluster of CTAs shares a head over distributed shared memory).  The row's
-// 16-cell tiles of one KV head are cut into kClWarps * kClCtas equal runs;
+// 16-cell tiles of one KV head are cut into kClWarps * kClCtas equal runs
+// (16 CTAs of 8 warps: one long row's 8 KV heads then cover 128 SMs);
 // each warp of each CTA of the cluster folds its run with the tensor-core
 // tile step (its own TMA ring, as in the stream kernel) and leaves its
 // partial (m, l, O) in its CTA's shared memory; after a cluster barrier CTA
@@ -416,7 +426,7 @@ int stream_blocks_per_sm() {
 // (rank, warp) order with the sink -- no workspace, no combine launch.  Both
 // cluster barriers are reached on every path (a warp whose bounded wait runs
 // out poisons its partial and drains its copies), so no CTA waits forever.
-constexpr int kClCtas = 8;    // CTAs per cluster (the portable maximum)
+constexpr int kClCtas = 16;   // CTAs per cluster (above the portable 8: opted in at launch)
 constexpr int kClWarps = 8;   // warps per CTA
 
 template <int D, int NH>
@@ -575,6 +585,16 @@ cudaError_t launch_cluster_t(const DecodePlan& p, const CUtensorMap& tmK, const 
   static std::atomic<unsigned long long> smem_set{0ull};
   cudaError_t e = set_smem_limit_once(smem_set, kern, Sm::TOTAL);
   if (e != cudaSuccess) return e;
+  static std::atomic<unsigned long long> np_set{0ull};
+  {
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(np_set.load() & bit)) {
+      if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess) return e;
+      np_set.fetch_or(bit);
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((int64_t)p.R * p.Hkv * kClCtas));
   cfg.blockDim = dim3(32 * kClWarps);

@@ -154,6 +154,10 @@ struct WarpTileState {
     if (kEarlyRelease) load_v(base);
   }
 
+  // (one-byte caches load per-cell scales ahead; 16-bit caches have none)
+  __device__ __forceinline__ void prefetch(const DecodePlan&, int, int, int) {}
+  __device__ __forceinline__ void take_prefetched() {}
+
   // Fold the loaded tile: cells tile0 .. tile0+15 of the row; only cells
   // < rc.s_end that pass the row filter count.
   __device__ __forceinline__ void compute(const DecodePlan& p, const RowCtx& rc, int r, int tile0,

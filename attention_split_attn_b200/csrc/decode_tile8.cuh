@@ -94,6 +94,24 @@ struct WarpTileState8 {
   uint32_t ka[KSTEPS][4];                    // K codes widened (A fragments of S^T)
   uint32_t vw[4][NB * 4];                    // V codes: this lane's 16-byte chunks of its 4 cells
   uint32_t koff[NB][2][2], voff[4][NB];      // shared-memory byte offsets inside a stage
+  // this lane's cells' K and V scales (cells grp, grp + 8): the current tile's,
+  // and the next tile's, loaded one tile ahead so their latency hides behind
+  // a tile's work
+  float cur_ks[2], cur_vs[2], nxt_ks[2], nxt_vs[2];
+
+  __device__ __forceinline__ void prefetch(const DecodePlan& p, int g, int tile0, int lane) {
+#pragma unroll
+    for (int kr = 0; kr < 2; ++kr) {
+      const int c = tile0 + (lane >> 2) + 8 * kr;
+      const int64_t si = (int64_t)c * p.scale_sc + g;
+      nxt_ks[kr] = c < p.N ? __ldg(p.k_scale + si) : 0.f;
+      nxt_vs[kr] = c < p.N ? __ldg(p.v_scale + si) : 0.f;
+    }
+  }
+  __device__ __forceinline__ void take_prefetched() {
+    cur_ks[0] = nxt_ks[0]; cur_ks[1] = nxt_ks[1];
+    cur_vs[0] = nxt_vs[0]; cur_vs[1] = nxt_vs[1];
+  }
 
   __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -262,9 +280,8 @@ struct WarpTileState8 {
         negdist = -(float)(rc.row_pos >= cpos ? rc.row_pos - cpos : cpos - rc.row_pos);
       }
       vis[kr] = vk;
-      const int64_t si = (int64_t)c * p.scale_sc + scale_head_;
-      const float ks = vk ? __ldg(p.k_scale + si) : 0.f;
-      vs[kr] = vk ? __ldg(p.v_scale + si) : 0.f;
+      const float ks = vk ? cur_ks[kr] : 0.f;
+      vs[kr] = vk ? cur_vs[kr] : 0.f;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll

@@ -87,7 +87,7 @@ cudaError_t launch_decode_slices(const DecodePlan& p, const CUtensorMap& tmK, co
 // Balanced persistent scheme: planner kernel, then W single-warp CTAs that
 // each take an equal run of the flattened (row, KV head, 16-cell tile) space.
 int decode_stream_warps(int kv_type, int D, int G, int sms);
-// Cluster decode (attn_decode_cluster): one 8-CTA cluster per (row, KV head),
+// Cluster decode (attn_decode_cluster): one 16-CTA cluster per (row, KV head),
 // partials folded over distributed shared memory; 16-bit caches, head dim
 // 64 or 128.
 cudaError_t launch_decode_cluster(const DecodePlan& p, const CUtensorMap& tmK, const CUtensorMap& tmV,

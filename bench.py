@@ -577,7 +577,7 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
 
     # one long row (130856 cached keys, the depth of TensorFold PR #2595's
     # long-context receipt), Hq 32 / Hkv 8, D 128, bf16: attn_decode (balanced
-    # kernel + split_k_reduce), attn_decode_cluster (8-CTA clusters, DSMEM
+    # kernel + split_k_reduce), attn_decode_cluster (16-CTA clusters, DSMEM
     # fold, no workspace) and attn_decode_append (the step's append fused in)
     p = W.random_problem(1010, R=1, Hq=32, Hkv=8, D=128, N=130857, kv_dtype=torch.bfloat16,
                          out_dtype=torch.bfloat16, lengths=[130857])
@@ -715,13 +715,35 @@ def run_profile_op(args, local):
         a = A.make_args(q, k, v, out, **kw)
         ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
         call = lambda: A.attn_decode_args(a, ws=ws)
-    elif op == "selected":
+    elif op in ("selected", "selected_masked"):
         p = W.selected_prefill()
         (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
         sel = kw.pop("sel")
         a = A.make_selected_args(q, k, v, out, sel, **kw)
-        ws = torch.empty(max(A.selected_workspace_size(a), 256), dtype=torch.uint8, device=dev)
-        call = lambda: A.attn_selected_args(a, ws=ws)
+        if op == "selected":
+            ws = torch.empty(max(A.selected_workspace_size(a), 256), dtype=torch.uint8, device=dev)
+            call = lambda: A.attn_selected_args(a, ws=ws)
+        else:
+            ws = torch.empty(max(A.selected_masked_workspace_size(a), 256), dtype=torch.uint8, device=dev)
+            call = lambda: A.attn_selected_masked_args(a, ws=ws)
+    elif op == "fp8":
+        p = W.quantized_decode(fmt="e4m3")
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_decode_args(a, ws=ws)
+    elif op == "tree":
+        p = W.tree_decode(width=16, visible=130856)
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_decode_args(a, ws=ws)
+    elif op == "long_row":
+        p = W.random_problem(1010, R=1, Hq=32, Hkv=8, D=128, N=130857, kv_dtype=torch.bfloat16,
+                             out_dtype=torch.bfloat16, lengths=[130857])
+        (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
+        a = A.make_args(q, k, v, out, **kw)
+        call = lambda: A.attn_decode_cluster_args(a)
     else:
         p = W.causal_prefill()
         (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
@@ -785,7 +807,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-parts", action="store_true", help="time the decode workload only")
-    ap.add_argument("--profile-op", choices=["decode", "selected", "prefill", "semantics"], default=None,
+    ap.add_argument("--profile-op", choices=["decode", "selected", "prefill", "semantics", "selected_masked", "fp8",
+                                             "tree", "long_row"], default=None,
                     help="only run W + K calls of one operation (for ncu captures); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup

@@ -235,15 +235,15 @@ int32_t attn_decode_append(const attn_args *args, const void *k_new, const void 
                            int64_t new_stride_head, void *ws, size_t ws_bytes, void *stream);
 
 /* attn_decode for few, long rows without a workspace: one thread-block
- * cluster of 8 CTAs per (row, KV head) (TensorFold PR #985, change list: a
+ * cluster of 16 CTAs per (row, KV head) (TensorFold PR #985, change list: a
  * cluster of CTAs shares a head over distributed shared memory).  Each of the
- * cluster's 64 warps folds an equal run of the row's 16-cell tiles on the
- * tensor cores; CTA rank 0 then reads the 64 partials over distributed shared
+ * cluster's 128 warps folds an equal run of the row's 16-cell tiles on the
+ * tensor cores; CTA rank 0 then reads the 128 partials over distributed shared
  * memory and folds them in order with the sink -- one launch, no workspace,
  * no split_k_reduce pass.  Same arguments and result as attn_decode (bit-
  * identical across runs); takes a 16-bit cache with Q in its dtype, head_dim
  * 64 or 128, up to 16 q heads per KV head, n_slices 0, no per-cell sequence
- * ids.  Intended for few rows (n_rows x n_head_kv clusters of 8 CTAs).     */
+ * ids.  Intended for few rows (n_rows x n_head_kv clusters of 16 CTAs).    */
 int32_t attn_decode_cluster(const attn_args *args, void *stream);
 
 /* The masked per-cell route of selected-key attention (strix-llama.cpp PR
