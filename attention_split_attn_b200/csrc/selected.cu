@@ -188,7 +188,10 @@ template <typename KT, int D, int NH>
 struct SelCfg {
   static constexpr int NW = D / 64;                   // warps (64 dims each)
   static constexpr int NT = NH / 8;                   // head n-tiles
-  static constexpr int RS = 64 * 2 + 16;              // row stride of a warp's slice (bytes)
+  // A warp's slice of a cell row is 128 bytes; rows are stored unpadded with
+  // 16-byte chunk k of row i at chunk k ^ (i & 7), so the 8 lanes copying one
+  // row and the 8 rows one ldmatrix reads both cover all 32 banks.
+  static constexpr int RS = 64 * 2;                   // row stride of a warp's slice (bytes)
   static constexpr int TILE_BYTES = kSelTile * RS;    // K or V slice of a block
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int NS = NW == 4 ? 2 : 3;          // ring stages per warp
@@ -253,8 +256,9 @@ selected_kernel(const SelectedPlan p) {
         const int c = __shfl_sync(0xffffffffu, cl, row);
         const bool valid = c >= 0;
         const int64_t off = (int64_t)(valid ? c : 0) * p.kv_sc + (int64_t)g * p.kv_sh + dw + chunk * 8;
-        cp_async16(st + row * C::RS + chunk * 16, kbase + off, valid);
-        cp_async16(st + C::TILE_BYTES + row * C::RS + chunk * 16, vbase + off, valid);
+        const uint32_t so = (uint32_t)(row * C::RS + ((chunk ^ (row & 7)) << 4));
+        cp_async16(st + so, kbase + off, valid);
+        cp_async16(st + C::TILE_BYTES + so, vbase + off, valid);
       }
     }
     cp_async_commit();
@@ -301,7 +305,7 @@ selected_kernel(const SelectedPlan p) {
       for (int kk = 0; kk < 4; ++kk) {
         const int row = mt * 16 + (lane & 7) + (mi & 1) * 8;
         const int chunk = 2 * kk + (mi >> 1);
-        koff[mt][kk] = row * C::RS + chunk * 16;
+        koff[mt][kk] = row * C::RS + ((chunk ^ (row & 7)) << 4);
       }
 #pragma unroll
     for (int m4 = 0; m4 < 4; ++m4)
@@ -309,7 +313,7 @@ selected_kernel(const SelectedPlan p) {
       for (int ks = 0; ks < 2; ++ks) {
         const int row = ks * 16 + (lane & 7) + (mi >> 1) * 8;
         const int chunk = 2 * m4 + (mi & 1);
-        voff[m4][ks] = C::TILE_BYTES + row * C::RS + chunk * 16;
+        voff[m4][ks] = C::TILE_BYTES + row * C::RS + ((chunk ^ (row & 7)) << 4);
       }
   }
 
