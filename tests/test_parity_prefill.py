@@ -155,11 +155,17 @@ def test_semantics_sweep_prefill(cuda_lib, semantics_problem):
 
 
 def test_causal_prefill_workload_sampled(cuda_lib):
-    """The full-size causal prefill workload; 24 sampled rows (all heads)
-    against the oracle, the first and last rows included."""
+    """The full-size causal prefill workload against the oracle on sampled
+    rows (all heads): one random row in every 128-row tile (so every unit of
+    the launch, split units included, is checked), both edges of the first
+    tile boundary, and the first and last rows."""
     p = W.causal_prefill()
     out = run_prefill(p)
     rng = np.random.default_rng(4)
-    rows = np.unique(np.concatenate([[0, p.n_rows - 1], rng.choice(p.n_rows, size=22, replace=False)]))
+    n_tiles = (p.n_rows + 127) // 128
+    per_tile = [t * 128 + int(rng.integers(min(128, p.n_rows - t * 128))) for t in range(n_tiles)]
+    rows = np.unique(np.concatenate([[0, 127, 128, p.n_rows - 1], per_tile,
+                                     rng.choice(p.n_rows, size=8, replace=False)]))
+    assert len(np.unique(rows // 128)) == n_tiles
     sub = p.row_subset(rows)
     check(sub, out[torch.from_numpy(rows).cuda()], "causal_prefill sample")
