@@ -130,11 +130,12 @@ CUtensorMapDataType tma_dtype(int32_t t) {
   }
 }
 
-// 3-D map over a [cells][heads][D] cache: box = (box_d, 1, box_cells); with
-// swizzle the box rows are 128 bytes and stored with the 128-byte swizzle.
+// 3-D map over a [cells][heads][D] cache: box = (box_d, box_heads, box_cells);
+// with swizzle the box rows are 128 bytes and stored with the 128-byte
+// swizzle (box row index = cell * box_heads + head).
 int32_t make_kv_map(CUtensorMap* map, const void* base, int32_t type, int D, int Hkv, int N,
                     int64_t stride_cell, int64_t stride_head, int box_cells, int box_d = 0,
-                    bool swizzle128 = false) {
+                    bool swizzle128 = false, int box_heads = 1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int es = dtype_size(type);
@@ -143,7 +144,7 @@ int32_t make_kv_map(CUtensorMap* map, const void* base, int32_t type, int D, int
   const int64_t sc = N > 1 ? stride_cell : D;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)N};
   cuuint64_t strides[2] = {(cuuint64_t)(sh * es), (cuuint64_t)(sc * es)};
-  cuuint32_t box[3] = {(cuuint32_t)(box_d > 0 ? box_d : D), 1u, (cuuint32_t)box_cells};
+  cuuint32_t box[3] = {(cuuint32_t)(box_d > 0 ? box_d : D), (cuuint32_t)box_heads, (cuuint32_t)box_cells};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(map, tma_dtype(type), 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -403,13 +404,23 @@ struct PrefillSplit {
   int64_t ctas() const { return n_full + n_split * k; }
 };
 
+// Packed rows: with fewer rows than a tile and several q heads per KV head,
+// a tile's 128 lanes hold 128 / G rows x the G heads of one KV group, so each
+// K and V tile is read once for all of them (draft-tree rows, short prefills).
+int32_t prefill_pack(const attn_args* a) {
+  const int G = a->n_head_q / a->n_head_kv;
+  return (G >= 2 && G <= kPfTile && a->n_rows < kPfTile) ? G : 1;
+}
+int32_t prefill_rows_per_tile(const attn_args* a) { return kPfTile / prefill_pack(a); }
+
 PrefillSplit plan_prefill_split(const attn_args* a, int sms) {
   PrefillSplit s{};
-  const int64_t n_rt = ((int64_t)a->n_rows + kPfTile - 1) / kPfTile;
+  const int rpt = prefill_rows_per_tile(a);
+  const int64_t n_rt = ((int64_t)a->n_rows + rpt - 1) / rpt;
   const int G = a->n_head_q / a->n_head_kv;
-  s.units = n_rt * a->n_head_kv * (a->head_dim <= 128 ? (G + 1) / 2 : G);
+  s.units = n_rt * a->n_head_kv * (prefill_pack(a) > 1 ? 1 : a->head_dim <= 128 ? (G + 1) / 2 : G);
   const int64_t r = s.units > sms ? s.units % sms : s.units;
-  const int64_t k = r > 0 ? std::min<int64_t>(4, sms / r) : 1;
+  const int64_t k = r > 0 ? std::min<int64_t>(32, sms / r) : 1;
   s.k = (int32_t)k;
   s.n_split = k >= 2 ? r : 0;
   s.n_full = s.units - s.n_split;
@@ -422,7 +433,8 @@ struct PrefillWs {
 };
 
 PrefillWs prefill_ws_layout(const attn_args* a, const PrefillSplit& sp) {
-  const size_t n_rt = ((size_t)a->n_rows + kPfTile - 1) / kPfTile;
+  const size_t rpt = (size_t)prefill_rows_per_tile(a);
+  const size_t n_rt = ((size_t)a->n_rows + rpt - 1) / rpt;
   const size_t n_kt = ((size_t)a->n_cells + kPfTile - 1) / kPfTile;
   PrefillWs w;
   w.vbad_off = align256(n_rt * n_kt);
@@ -908,9 +920,11 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   memset(&tmQ, 0, sizeof(tmQ));
   memset(&tmK, 0, sizeof(tmK));
   memset(&tmV, 0, sizeof(tmV));
-  // Q as a [rows][heads][D] array with 128-row boxes; K and V with 128-cell boxes.
+  // Q as a [rows][heads][D] array with boxes of 128 rows of one head (packed:
+  // 128 / G rows of the G heads of a KV group); K and V with 128-cell boxes.
+  const int32_t pack = prefill_pack(a), rpt = prefill_rows_per_tile(a);
   if ((st = make_kv_map(&tmQ, a->q, a->q_type, a->head_dim, a->n_head_q, a->n_rows, a->q_stride_row,
-                        a->q_stride_head, kPfTile, 64, true)) != ATTN_OK)
+                        a->q_stride_head, rpt, 64, true, pack)) != ATTN_OK)
     return st;
   if (a->n_cells > 0) {
     if ((st = make_kv_map(&tmK, a->k, a->kv_type, a->head_dim, a->n_head_kv, a->n_cells, a->kv_stride_cell,
@@ -929,9 +943,12 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   p.f = RowFilter{a->row_begin, a->row_end, a->cell_seq, a->row_seq, a->cell_pos, a->row_pos,
                   a->causal, a->mask, a->mask_stride_row};
   p.lg = Logits{a->scale, a->softcap, a->alibi_slopes, a->sinks};
-  p.n_rt = (a->n_rows + kPfTile - 1) / kPfTile;
+  p.pack = pack;
+  p.rpt = rpt;
+  p.n_rt = (a->n_rows + rpt - 1) / rpt;
   p.n_kt = (a->n_cells + kPfTile - 1) / kPfTile;
-  p.n_pairs = a->head_dim <= 128 ? (p.G + 1) / 2 : p.G;   // q heads per CTA: 2 up to head dim 128, 1 at 256
+  // q heads per CTA: 2 up to head dim 128, 1 at 256; packed: all G in one slot
+  p.n_pairs = pack > 1 ? 1 : a->head_dim <= 128 ? (p.G + 1) / 2 : p.G;
   char* wsb = static_cast<char*>(ws);
   p.cls = reinterpret_cast<uint8_t*>(wsb);
   p.vbad = reinterpret_cast<uint8_t*>(wsb + wl.vbad_off);

@@ -157,7 +157,13 @@ struct PrefillPlan {
   RowFilter f;
   Logits lg;
   int32_t n_rt, n_kt;       // row tiles, cell tiles (128 each)
-  int32_t n_pairs;          // CTAs per (row tile, KV head): ceil(G / 2) up to head dim 128, G at 256
+  int32_t n_pairs;          // CTAs per (row tile, KV head): ceil(G / 2) up to head dim 128, G at 256 (1 packed)
+  // Packed rows (pack > 1, fewer rows than a tile): the 128 lanes of a tile
+  // hold rpt = 128 / pack rows x the pack = G q heads of one KV group (lane
+  // t: row t / pack, head t % pack), so every K and V tile serves all of the
+  // group's heads at once; one CTA per (row tile, KV head).  Else pack = 1,
+  // rpt = 128.
+  int32_t pack, rpt;
   uint8_t* cls;             // workspace [n_rt][n_kt]
   uint32_t* bits;           // workspace [n_rt][n_kt][128 rows][4 words] (with a mask) or NULL
   uint8_t* vbad;            // workspace [n_kt][Hkv]

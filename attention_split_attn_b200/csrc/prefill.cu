@@ -18,6 +18,11 @@
 //    paths: strix-llama.cpp PR #115 "Performance" discussion.)
 //  * prefill_kernel: one CTA per (row tile, two q heads of one KV group).  Both
 //    heads share every K and V tile, so each tile crosses L2 once per pair.
+//    With fewer rows than a tile and several q heads per KV head (draft-tree
+//    rows, short prefills) the rows are packed: a tile's 128 lanes hold
+//    128 / G rows x the G heads of one KV group (lane t: row t / G, head
+//    t % G, the Q box being G heads x 128 / G rows), one head slot per CTA,
+//    so each K and V tile serves the whole group at once.
 //      warp 0       TMA producer: Q of both heads once, then K_j into a
 //                   one-tile K buffer and V_j into a two-tile V ring
 //                   (128-byte swizzled boxes of 64 x 128).
@@ -80,8 +85,9 @@ __device__ __forceinline__ RowVis row_vis(const RowFilter& f, int r, int N) {
   return v;
 }
 
-// Classification of tile b = (rt, kt) by one CTA of 256 threads: the 128
-// rows' range, sequence and position are staged in shared memory; warp w
+// Classification of tile b = (rt, kt) by one CTA of 256 threads: the tile's
+// rows' (128, or 128 / G when rows are packed) range, sequence and position
+// are staged in shared memory; warp w
 // takes rows w, w + 8, ..., lane l cells 4l .. 4l + 3 of the tile, and each
 // warp issues its 16 rows' 16-byte mask loads before using any of them (the
 // scan is bound by DRAM latency otherwise).  A row's visibility bits are gathered from the lanes'
@@ -92,8 +98,8 @@ constexpr int kClsRowsPerWarp = kPfRows / (kClsThreads / 32);   // 16
 __device__ __forceinline__ void pf_classify_tile(const PrefillPlan& p, int64_t b, int4* rows_sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rt = (int)(b / p.n_kt), kt = (int)(b % p.n_kt);
-    if (tid < kPfRows) {
-      const int r = rt * kPfRows + tid;
+    if (tid < p.rpt) {
+      const int r = rt * p.rpt + tid;
       const RowVis rv = r < p.R ? row_vis(p.f, r, p.N) : RowVis{0, 0, 0, 0};
       rows_sh[tid] = make_int4(rv.rb, rv.re, rv.rs, rv.rp);
     }
@@ -112,9 +118,9 @@ __device__ __forceinline__ void pf_classify_tile(const PrefillPlan& p, int64_t b
       const bool vec = p.mask_vec && kt * kPfCells + kPfCells <= p.N;
 #pragma unroll
       for (int i = 0; i < kClsRowsPerWarp; ++i) {
-        const int r = rt * kPfRows + warp + 8 * i;
+        const int r = rt * p.rpt + warp + 8 * i;
         mv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < p.R) {
+        if (warp + 8 * i < p.rpt && r < p.R) {
           const float* mrow = p.f.mask + (int64_t)r * p.f.mask_sr + c_base;
           if (vec) {
             mv[i] = __ldg(reinterpret_cast<const float4*>(mrow));
@@ -132,7 +138,7 @@ __device__ __forceinline__ void pf_classify_tile(const PrefillPlan& p, int64_t b
 #pragma unroll
     for (int i = 0; i < kClsRowsPerWarp; ++i) {
       const int rl = warp + 8 * i;
-      if (rt * kPfRows + rl >= p.R) continue;   // warp-uniform
+      if (rl >= p.rpt || rt * p.rpt + rl >= p.R) continue;   // warp-uniform
       const int4 rv = rows_sh[rl];
       const float mvals[4] = {mv[i].x, mv[i].y, mv[i].z, mv[i].w};
       uint32_t nib = 0u;
@@ -282,7 +288,8 @@ struct PfLayout {
   static constexpr int OFF_V = OFF_K + NK * TILE;        // [NV][TILE]
   static constexpr int OFF_BAR = OFF_V + NV * TILE;
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
-  // p_full[2], pv_done[2], mma_done, stall (never arrived at: the bounded-wait test)
+  // p_full[2], pv_last[2] (the last P V of each head slot), mma_done, stall
+  // (never arrived at: the bounded-wait test)
   static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 6 + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;   // TMEM base address, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
@@ -315,7 +322,7 @@ template <int N>
 __device__ __forceinline__ uint32_t pf_phase(int64_t i) { return (uint32_t)((i / N) & 1); }
 
 struct PfBars {
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *pv_done, *mma_done, *stall;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *pv_last, *mma_done, *stall;
 };
 template <int D>
 __device__ __forceinline__ PfBars pf_bars(unsigned char* sm) {
@@ -329,7 +336,7 @@ __device__ __forceinline__ PfBars pf_bars(unsigned char* sm) {
   r.v_empty = r.v_full + L::NV;
   r.s_full = r.v_empty + L::NV;
   r.p_full = r.s_full + 2;
-  r.pv_done = r.s_full + 4;
+  r.pv_last = r.s_full + 4;   // [2]: the last P V of each head slot retired
   r.mma_done = r.s_full + 6;
   r.stall = r.s_full + 7;
   return r;
@@ -783,8 +790,8 @@ __device__ __forceinline__ void pf_pv_cuda_cores(const uint32_t* pk, const uint3
 #pragma unroll
     for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e]);
     tmem_st32(tO + ch * 32, ou);
+    tmem_wait_st();
   }
-  tmem_wait_st();
 }
 
 // A CTA's share of a split unit: part `part` of nparts; su = the unit's index
@@ -868,15 +875,15 @@ __device__ __noinline__ void pf_split_epilogue(const PrefillPlan& p, const PfSpl
   }
 }
 
-template <typename KT, int D>
+template <typename KT, int D, bool PK>
 __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& tiles, unsigned char* sm,
                                            const PfBars& B, volatile int* abort_flag, uint32_t tmem, int rt,
                                            int h, int slot, int quarter, int lane, const PfSplit& split) {
+  // (h: this slot's q head; with packed rows, the KV group's first head)
   const bool out_vec = p.out_vec != 0, mask_vec = p.mask_vec != 0;
   using L = PfLayout<D>;
   uint64_t* s_full = B.s_full;
   uint64_t* p_full = B.p_full;
-  uint64_t* pv_done = B.pv_done;
   // Bounded-wait test: wait on a barrier nothing arrives at; the wait gives
   // up after p.wait_ns, records the timeout and raises the abort flag, and
   // every role of the CTA then winds down.
@@ -884,8 +891,14 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     if (!pf_wait_warp(B.stall, 0u, p, abort_flag)) return;
   }
   const int row_t = quarter * 32 + lane;
-  const int r = rt * kPfRows + row_t;
-  const bool rvalid = r < p.R;
+  // packed rows: lane row_t holds row row_t / pack of the tile, head
+  // h + row_t % pack (h is then the KV group's first head)
+  // (PK: the launch has packed rows; the unpacked kernel compiles without them)
+  const int pack = PK ? p.pack : 1, rpt = PK ? p.rpt : kPfRows;
+  const int row_l = PK ? row_t / pack : row_t;
+  if (PK) h += row_t % pack;
+  const int r = rt * rpt + row_l;
+  const bool rvalid = (!PK || row_t < pack * rpt) && r < p.R;
   const RowVis rv = rvalid ? row_vis(p.f, r, p.N) : RowVis{0, 0, 0, 0};
   const bool alibi = p.lg.slopes != nullptr;
   const float nslope = alibi ? -__ldg(p.lg.slopes + h) : 0.f;
@@ -960,7 +973,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
           int i_lo = 0, i_hi = kPfCells - 1;
           if (bits_tile) {
             const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
-                                          p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_t) << 2)))
+                                          p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_l) << 2)))
                                     : make_uint4(0u, 0u, 0u, 0u);
             vis[0] = bw.x; vis[1] = bw.y; vis[2] = bw.z; vis[3] = bw.w;
             i_hi = vis[3] ? 96 + 31 - __clz(vis[3]) : vis[2] ? 64 + 31 - __clz(vis[2])
@@ -1035,7 +1048,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
         const float boff = al == 1 ? C : 0.f, bstep = al == 1 ? 8.f * slope : 0.f;
         if (bits_tile) {
           const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
-                                        p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_t) << 2)))
+                                        p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_l) << 2)))
                                   : make_uint4(0u, 0u, 0u, 0u);
           vis[0] = bw.x; vis[1] = bw.y; vis[2] = bw.z; vis[3] = bw.w;
           pf_apply_bits(x, vis, boff, bstep, mt);
@@ -1090,8 +1103,8 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
           o[e + 1] = __float_as_uint(v.y);
         }
         tmem_st32(tO + ch * 32, o);
+        tmem_wait_st();
       }
-      tmem_wait_st();
     }
 
     if (code == kTileMixedBadV) {
@@ -1112,7 +1125,10 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
 
   if (!ok) return;
   if (j > 0) {
-    if (!pf_wait_warp(&pv_done[slot], (uint32_t)((j - 1) & 1), p, abort_flag)) return;
+    // the last P V of this head: a barrier with one phase per launch, so the
+    // wait is exact (a parity wait on a barrier that completed a phase per
+    // tile and was never waited for before could pass early)
+    if (!pf_wait_warp(&B.pv_last[slot], 0u, p, abort_flag)) return;
     tc_fence_after();
   }
   if (split.nparts > 1) {
@@ -1153,7 +1169,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
 
 // One CTA per (row tile, KV head g, pair of q heads of g).  Heavier row tiles
 // (later rows see more cells under causality) are launched first.
-template <typename KT, int D>
+template <typename KT, int D, bool PK>
 __global__ void __launch_bounds__(PfLayout<D>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const PrefillPlan p) {
@@ -1180,7 +1196,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int g = (int)(unit % per_rt) / p.n_pairs;
   const int pair = (int)(unit % per_rt) % p.n_pairs;
   const int h0 = g * p.G + L::HPC * pair;
-  const int n_slots = min(L::HPC, p.G - L::HPC * pair);
+  // packed rows: one slot holding all of the group's heads
+  const int n_slots = PK ? 1 : min(L::HPC, p.G - L::HPC * pair);
+  const int rpt = PK ? p.rpt : kPfRows;
+  // bytes of a slot's Q tile as loaded: rpt rows x pack heads x D
+  const uint32_t q_bytes = PK ? (uint32_t)(p.rpt * p.pack) * (uint32_t)(D * 2) : (uint32_t)L::TILE;
 
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 1);
@@ -1189,7 +1209,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.s_full[s], 1);
       mbar_init(&B.p_full[s], kPfRows);
-      mbar_init(&B.pv_done[s], 1);
+      mbar_init(&B.pv_last[s], 1);
     }
     mbar_init(B.mma_done, 1);
     mbar_init(B.stall, 1);
@@ -1197,6 +1217,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, L::TMEM_COLS);
+  if (PK && p.pack * p.rpt < kPfRows) {
+    // packed rows that leave lanes unused: zero those rows of the Q tile
+    // (its load writes the others), so the unused lanes of S stay finite
+    const int used = p.pack * p.rpt;
+    for (int i = threadIdx.x; i < (kPfRows - used) * (D / 8); i += L::THREADS) {
+      const int row = used + i % (kPfRows - used), chunk = i / (kPfRows - used);   // chunk: 16 bytes of D
+      *reinterpret_cast<uint4*>(sm + L::OFF_Q + (chunk >> 3) * L::BOX + row * 128 + (chunk & 7) * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();   // visible to the tensor core
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1238,7 +1269,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     setmaxnreg_inc<L::HIGH_REGS>();
     const int slot = (warp >> 2) - 1;
     if (slot < n_slots)
-      pf_softmax<KT, D>(p, tiles, sm, B, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane, split);
+      pf_softmax<KT, D, PK>(p, tiles, sm, B, abort_flag, tmem, rt, h0 + slot, slot, warp & 3, lane, split);
   } else {
   setmaxnreg_dec<L::LOW_REGS>();
   if (warp == 0) {
@@ -1250,11 +1281,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int64_t nK = 0, nV = 0;
       const bool any = kt >= 0;
       if (any) {
-        mbar_arrive_expect_tx(B.q_full, (uint32_t)(n_slots * L::TILE));
+        mbar_arrive_expect_tx(B.q_full, (uint32_t)n_slots * q_bytes);
         for (int s = 0; s < n_slots; ++s)
 #pragma unroll
           for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, B.q_full, bx * 64, h0 + s, rt * kPfRows,
+            tma_load_3d(sm + L::OFF_Q + s * L::TILE + bx * L::BOX, &tmQ, B.q_full, bx * 64, h0 + s, rt * rpt,
                         pol);
       }
       for (; kt >= 0; kt = tiles.next(kt)) {
@@ -1324,7 +1355,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (pv_mma)
             pf_issue_pv_ts<D>(tmem + 256u + (uint32_t)s * D, tmem + (uint32_t)s * 128u,
                               v_desc + (uint64_t)stV * kTileDesc, idO, j > 0);
-          umma_commit(&B.pv_done[s]);
+          if (!has_next) umma_commit(&B.pv_last[s]);
           if (has_next) {
             if (s == 0 && !pf_wait(&B.k_full[stK], pf_phase<NK>(j + 1), p, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -1352,11 +1383,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
 }
 
-template <typename KT, int D>
+template <typename KT, int D, bool PK>
 cudaError_t launch_prefill_t(const PrefillPlan& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, cudaStream_t stream, cudaEvent_t after_classify) {
   using L = PfLayout<D>;
-  auto kern = prefill_kernel<KT, D>;
+  auto kern = prefill_kernel<KT, D, PK>;
   static std::atomic<unsigned long long> smem_set{0ull};
   cudaError_t e = set_smem_limit_once(smem_set, kern, L::SMEM);
   if (e != cudaSuccess) return e;
@@ -1389,13 +1420,19 @@ cudaError_t launch_prefill(const PrefillPlan& p, const CUtensorMap& tmQ, const C
                            const CUtensorMap& tmV, cudaStream_t stream, cudaEvent_t after_classify) {
   const bool bf = p.kv_type == ATTN_BF16;
   if (p.D == 64)
-    return bf ? launch_prefill_t<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, stream, after_classify)
-              : launch_prefill_t<__half, 64>(p, tmQ, tmK, tmV, stream, after_classify);
+    return bf ? (p.pack > 1 ? launch_prefill_t<__nv_bfloat16, 64, true>(p, tmQ, tmK, tmV, stream, after_classify)
+                         : launch_prefill_t<__nv_bfloat16, 64, false>(p, tmQ, tmK, tmV, stream, after_classify))
+              : (p.pack > 1 ? launch_prefill_t<__half, 64, true>(p, tmQ, tmK, tmV, stream, after_classify)
+                         : launch_prefill_t<__half, 64, false>(p, tmQ, tmK, tmV, stream, after_classify));
   if (p.D == 256)
-    return bf ? launch_prefill_t<__nv_bfloat16, 256>(p, tmQ, tmK, tmV, stream, after_classify)
-              : launch_prefill_t<__half, 256>(p, tmQ, tmK, tmV, stream, after_classify);
-  return bf ? launch_prefill_t<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, stream, after_classify)
-            : launch_prefill_t<__half, 128>(p, tmQ, tmK, tmV, stream, after_classify);
+    return bf ? (p.pack > 1 ? launch_prefill_t<__nv_bfloat16, 256, true>(p, tmQ, tmK, tmV, stream, after_classify)
+                         : launch_prefill_t<__nv_bfloat16, 256, false>(p, tmQ, tmK, tmV, stream, after_classify))
+              : (p.pack > 1 ? launch_prefill_t<__half, 256, true>(p, tmQ, tmK, tmV, stream, after_classify)
+                         : launch_prefill_t<__half, 256, false>(p, tmQ, tmK, tmV, stream, after_classify));
+  return bf ? (p.pack > 1 ? launch_prefill_t<__nv_bfloat16, 128, true>(p, tmQ, tmK, tmV, stream, after_classify)
+                         : launch_prefill_t<__nv_bfloat16, 128, false>(p, tmQ, tmK, tmV, stream, after_classify))
+            : (p.pack > 1 ? launch_prefill_t<__half, 128, true>(p, tmQ, tmK, tmV, stream, after_classify)
+                         : launch_prefill_t<__half, 128, false>(p, tmQ, tmK, tmV, stream, after_classify));
 }
 
 }  // namespace attn

@@ -532,7 +532,10 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
 
     # draft-tree decode rows: 16 nodes of a binary draft tree over 130856 keys
     # (the depth of TensorFold PR #2595's long-context receipt), GQA heads;
-    # a call = the tree mask kernel + attn_decode.  Algorithmic bytes: the K/V
+    # a call = the tree mask kernel + attn_prefill, whose tiles then hold the
+    # 16 rows x the 4 q heads of a KV group (packed rows), so each K/V tile
+    # is read once for all of them; the same rows through attn_decode (each
+    # row streams the prefix) are timed beside it.  Algorithmic bytes: the K/V
     # rows of every cell some row sees, once (the rows share the prefix), the
     # mask, Q and the output; rows_per_s and the per-row view are beside it.
     p = W.tree_decode(width=16, visible=130856)
@@ -542,29 +545,39 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
     tmask = torch.empty((p.n_rows, p.n_cells), dtype=torch.float32, device=dev)
     ta = A.make_args(q, k, v, out, mask=tmask, **kw)
     ws = torch.empty(max(A.workspace_size(ta, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
+    wsp = torch.empty(max(A.workspace_size(ta, A.OP_PREFILL), 256), dtype=torch.uint8, device=dev)
     vis = int(torch.isfinite(p.mask).sum())
     cells = int(torch.isfinite(p.mask).any(dim=0).sum())
     kv_cell = p.n_head_kv * p.head_dim * p.k.element_size() * 2
     rest = p.n_rows * p.n_cells * 4 + p.q.numel() * p.q.element_size() + p.n_rows * p.n_head_q * p.head_dim * 2
     tbytes = cells * kv_cell + rest
 
-    def tree_call(e):
+    def tree_call_decode(e):
         e[0].record(stream)
         A.tree_mask(parent, p.tree_prefix, p.n_cells, mask=tmask, stream=stream)
         A.attn_decode_args(ta, ws=ws, stream=stream)
         e[1].record(stream)
         e[2].record(stream)
 
+    def tree_call(e):
+        e[0].record(stream)
+        A.tree_mask(parent, p.tree_prefix, p.n_cells, mask=tmask, stream=stream)
+        A.attn_prefill_args(ta, ws=wsp, stream=stream)
+        e[1].record(stream)
+        e[2].record(stream)
+
     for _ in range(max(args.warmup, 3)):
+        tree_call_decode([torch.cuda.Event(enable_timing=True) for _ in range(3)])
         tree_call([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    whole_dec, _ = _time_calls(tree_call_decode, n, flush, stream)
     whole, main = _time_calls(tree_call, n, flush, stream)
     parts["tree_decode"] = {
         "workload": "tree_decode: 16 draft-tree rows (binary heap order) over 130856 keys, Hq 32 / Hkv 8, D 128, "
-                    "bf16 KV and out; tree mask + attn_decode",
+                    "bf16 KV and out; tree mask + attn_prefill (packed rows)",
         "value": tbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (K/V of every visible cell once + mask)",
         "per_row_GBs": (vis * kv_cell + rest) / (whole * 1e-3) / 1e9,
-        "ms_per_call": whole, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
-        "gpu_launches": 3 * n,   # tree mask + stream kernel + split_k_reduce
+        "ms_per_call": whole, "ms_attn_decode": whole_dec, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
+        "gpu_launches": 3 * n,   # tree mask + classifier + tensor-core kernel
         "roofline": {"bound": "hbm", "achieved": tbytes / (main * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": tbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None, "kernel_ms": main,
                      "algorithmic_bytes": tbytes,

@@ -30,10 +30,16 @@
  *                  PV.  Supported: K/V and Q in F16 or BF16 (same dtype),
  *                  head_dim 64, 128 or 256, Q 16-byte aligned with strides
  *                  that are multiples of 16 bytes; any out dtype.  n_slices,
- *                  max_row_len and grid_order are ignored.  Workspace: one
- *                  byte per (128-row tile, 128-cell tile) and per (cell tile,
- *                  KV head), plus the visibility bits of every tile when a
- *                  mask is given.
+ *                  max_row_len and grid_order are ignored.  With fewer than
+ *                  128 rows and G >= 2 query heads per KV head (draft-tree
+ *                  rows, short prefills) a tile's 128 rows hold 128 / G
+ *                  query rows x the G heads of one KV group, so each K/V
+ *                  tile is read once for the whole group; few work units
+ *                  are split into up to 32 parts over their cell tiles.
+ *                  Workspace: one byte per (row tile, 128-cell tile) and per
+ *                  (cell tile, KV head), the visibility bits of every tile
+ *                  when a mask is given, and the split parts' partial
+ *                  results (attn_workspace_size gives the total).
  *
  * Unified caches.  When cell_seq/row_seq are given (several sequences'
  * cells interleaved in one cache, strix-llama.cpp PR #115 "Isolation"), the
