@@ -296,7 +296,7 @@ def run_ours(args, rank, world, local):
     main_ms = [e[0].elapsed_time(e[1]) for e in ev]
     kmean_ms = sum(main_ms) / len(main_ms)
     achieved = step_bytes / (kmean_ms * 1e-3) / 1e9
-    traffic = _recorded_traffic("decode_stream_kernel")
+    traffic = _recorded_traffic("gqa_decode")
 
     e2e = run_e2e(args, sets, stream)
     with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -338,15 +338,16 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-def _recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary
-    (profiles/traffic.json), if it was taken on the current sources (else None)."""
+def _recorded_traffic(part: str):
+    """DRAM bytes per launch of the dominant kernel of bench part `part` from
+    the committed ncu summary (profiles/traffic.json), if it was taken on the
+    current sources of that kernel (else None)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f).get(kernel)
+        d = json.load(f).get(part)
     if not d:
         return None
     m = hashlib.sha256()
@@ -468,7 +469,7 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
         "gpu_launches": 2 * n,
         "roofline": {"bound": "hbm", "achieved": nbytes / (main * 1e-3) / 1e9, "peak": hbm_peak,
                      "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak,
-                     "traffic": _recorded_traffic("selected_kernel"),
+                     "traffic": _recorded_traffic("selected"),
                      "kernel": "select_bitmap_kernel + selected_kernel",
                      "kernel_ms": main, "algorithmic_bytes": nbytes,
                      "peak_kind": f"{peak_kind} hbm_gbs (burst copy); gathered rows are mostly L2 hits"},
@@ -496,7 +497,7 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
         "ms_per_call": whole_m, "vs_selected_kernel": whole_m / whole, "calls": nm,
         "gpu_launches": 3 * nm,   # mask builder + tile classifier + tensor-core kernel
         "roofline": {"bound": "tensor", "achieved": sflops / (main_m * 1e-3) / 1e12, "peak": tc_peak,
-                     "unit": "TFLOP/s", "frac": sflops / (main_m * 1e-3) / 1e12 / tc_peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": sflops / (main_m * 1e-3) / 1e12 / tc_peak, "traffic": _recorded_traffic("selected_masked"),
                      "kernel": "sel_mask_kernel + prefill_classify_kernel + prefill_kernel<f16, 256>",
                      "kernel_ms": main_m, "algorithmic_flops": sflops,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS); flops of the selected pairs only"},
@@ -520,7 +521,7 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
         "gpu_launches": 2 * n,
         "roofline": {"bound": "tensor", "achieved": flops / (main * 1e-3) / 1e12, "peak": tc_peak,
                      "unit": "TFLOP/s", "frac": flops / (main * 1e-3) / 1e12 / tc_peak,
-                     "traffic": _recorded_traffic("prefill_kernel"),
+                     "traffic": _recorded_traffic("prefill"),
                      "kernel": "prefill_classify_kernel + prefill_kernel (tcgen05)",
                      "kernel_ms": main, "algorithmic_flops": flops,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS)"},
@@ -579,9 +580,9 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
         "ms_per_call": whole, "ms_attn_decode": whole_dec, "rows_per_s": p.n_rows / (whole * 1e-3), "calls": n,
         "gpu_launches": 3 * n,   # tree mask + classifier + tensor-core kernel
         "roofline": {"bound": "hbm", "achieved": tbytes / (main * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": tbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None, "kernel_ms": main,
+                     "frac": tbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": _recorded_traffic("tree_decode"), "kernel_ms": main,
                      "algorithmic_bytes": tbytes,
-                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy); each row streams the shared prefix"},
+                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy); K/V of the tree's KV groups read once"},
     }
     if with_cpu:
         parts["tree_decode"]["cpu_baseline"] = _part_baseline(
@@ -623,7 +624,7 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
         "GBs_attn_decode": lbytes / (lat["decode"] * 1e-3) / 1e9, "calls": n,
         "gpu_launches": n * (1 + 2 + 2),   # cluster; decode (stream + combine); append (stream + combine)
         "roofline": {"bound": "hbm", "achieved": lbytes / (lat["cluster"] * 1e-3) / 1e9, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": lbytes / (lat["cluster"] * 1e-3) / 1e9 / hbm_peak, "traffic": None,
+                     "unit": "GB/s", "frac": lbytes / (lat["cluster"] * 1e-3) / 1e9 / hbm_peak, "traffic": _recorded_traffic("long_row_decode"),
                      "kernel": "decode_cluster_kernel (one launch)", "kernel_ms": lat["cluster"],
                      "algorithmic_bytes": lbytes, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
     }
@@ -649,9 +650,9 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
                     "F32 scales, len U[1024,8192], bf16 out",
         "value": qbytes / (whole * 1e-3) / 1e9, "unit": "GB/s (visible K/V codes + scales, Q, out)",
         "ms_per_call": whole, "calls": n,
-        "gpu_launches": (2 if qws_n > 0 else 1) * n,   # slice kernel (+ split_k_reduce)
+        "gpu_launches": (2 if qws_n > 0 else 1) * n,   # decode kernel (+ split_k_reduce)
         "roofline": {"bound": "hbm", "achieved": qbytes / (main * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": qbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None, "kernel_ms": main,
+                     "frac": qbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": _recorded_traffic("fp8_decode"), "kernel_ms": main,
                      "algorithmic_bytes": qbytes,
                      "kernel": "decode_stream_kernel<e4m3> (codes widened to f16 for the tensor cores) + combine_kernel",
                      "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
@@ -687,7 +688,7 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
             # visible lists + gather + split_k_reduce (long rows are split into parts)
             "gpu_launches": 3 * n,
             "roofline": {"bound": "hbm", "achieved": nbytes / (main * 1e-3) / 1e9, "peak": hbm_peak,
-                         "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": None,
+                         "unit": "GB/s", "frac": nbytes / (main * 1e-3) / 1e9 / hbm_peak, "traffic": _recorded_traffic("semantics"),
                          "kernel_ms": main, "algorithmic_bytes": nbytes,
                          "peak_kind": f"{peak_kind} hbm_gbs (burst copy); semantics case, no target"},
         }
@@ -746,11 +747,12 @@ def run_profile_op(args, local):
         ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
         call = lambda: A.attn_decode_args(a, ws=ws)
     elif op == "tree":
+        # the bench's tree rows: the host-built tree mask, attn_prefill (packed rows)
         p = W.tree_decode(width=16, visible=130856)
         (q, k, v, out), kw = A.problem_kwargs(p, device=dev)
         a = A.make_args(q, k, v, out, **kw)
-        ws = torch.empty(max(A.workspace_size(a, A.OP_DECODE), 256), dtype=torch.uint8, device=dev)
-        call = lambda: A.attn_decode_args(a, ws=ws)
+        ws = torch.empty(max(A.workspace_size(a, A.OP_PREFILL), 256), dtype=torch.uint8, device=dev)
+        call = lambda: A.attn_prefill_args(a, ws=ws)
     elif op == "long_row":
         p = W.random_problem(1010, R=1, Hq=32, Hkv=8, D=128, N=130857, kv_dtype=torch.bfloat16,
                              out_dtype=torch.bfloat16, lengths=[130857])
