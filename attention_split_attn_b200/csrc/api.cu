@@ -174,8 +174,8 @@ int32_t validate_common(const attn_args* a, int32_t op) {
   if (is_quantized(a->q_type) || is_quantized(a->out_type))
     return fail(ATTN_ERR_UNSUPPORTED, "Q and out cannot be e4m3 or int8 (only the K/V cache can)");
   if (is_quantized(a->kv_type)) {
-    if (op != ATTN_OP_DECODE)
-      return fail(ATTN_ERR_UNSUPPORTED, "e4m3/int8 K/V caches are supported by attn_decode only");
+    if (op != ATTN_OP_DECODE && op != ATTN_OP_PREFILL)
+      return fail(ATTN_ERR_UNSUPPORTED, "e4m3/int8 K/V caches are supported by attn_decode and attn_prefill only");
     if (a->n_cells > 0 && (!a->k_scale || !a->v_scale))
       return fail(ATTN_ERR_INVALID_ARG, "an e4m3/int8 cache needs k_scale and v_scale");
     if (a->n_cells > 1 && a->scale_stride_cell < a->n_head_kv)
@@ -368,9 +368,18 @@ bool unified_route(const attn_args* a);
 int32_t check_prefill(const attn_args* a) {
   int32_t st = validate_common(a, ATTN_OP_PREFILL);
   if (st != ATTN_OK) return st;
-  if (a->kv_type != ATTN_F16 && a->kv_type != ATTN_BF16)
-    return fail(ATTN_ERR_UNSUPPORTED, "prefill: K/V must be F16 or BF16");
-  if (a->q_type != a->kv_type) return fail(ATTN_ERR_UNSUPPORTED, "prefill: Q must be in the K/V dtype");
+  if (is_quantized(a->kv_type)) {
+    // codes widened to the Q dtype in the workspace, then the 16-bit path
+    if (a->q_type != ATTN_F16 && a->q_type != ATTN_BF16)
+      return fail(ATTN_ERR_UNSUPPORTED, "prefill over an e4m3/int8 cache: Q must be F16 or BF16");
+    if (a->n_cells > 0 && (!aligned16(a->k) || !aligned16(a->v) ||
+                           (a->n_cells > 1 && a->kv_stride_cell % 16) || (a->n_head_kv > 1 && a->kv_stride_head % 16)))
+      return fail(ATTN_ERR_UNSUPPORTED, "prefill over an e4m3/int8 cache: K/V and their strides 16-byte aligned");
+  } else {
+    if (a->kv_type != ATTN_F16 && a->kv_type != ATTN_BF16)
+      return fail(ATTN_ERR_UNSUPPORTED, "prefill: K/V must be F16 or BF16");
+    if (a->q_type != a->kv_type) return fail(ATTN_ERR_UNSUPPORTED, "prefill: Q must be in the K/V dtype");
+  }
   if (a->head_dim != 64 && a->head_dim != 128 && a->head_dim != 256)
     return fail(ATTN_ERR_UNSUPPORTED, "prefill: head_dim %d not in {64, 128, 256}", a->head_dim);
   if (a->reserved[0] < 0 || a->reserved[0] > 1000000)
@@ -395,7 +404,7 @@ int32_t check_prefill(const attn_args* a) {
 // Work units of the tensor-core kernel: (row tile, KV head, q heads per CTA),
 // heaviest row tiles first.  The units of a last, partial wave over the SMs
 // (or every unit, when there are fewer units than SMs) are split into k
-// parts over their cell tiles, k = SMs / (those units) clamped to 2..4, so
+// parts over their cell tiles, k = SMs / (those units) clamped to 2..32, so
 // the last wave holds shorter pieces; the parts' (m, l, O) are folded by the
 // last part to finish.
 struct PrefillSplit {
@@ -594,6 +603,37 @@ int32_t check_selected_masked(const attn_args* b) {
   return check_prefill(&pa);
 }
 
+// Prefill over an e4m3 / int8 cache: K and V widened to F16 (code x scale,
+// rounded once) into two contiguous [n_cells][n_head_kv][head_dim] arrays at
+// the start of the workspace, and a BF16 Q copied to F16 after them (the
+// tensor cores take both operands in one type); the prefill then runs on
+// these copies.
+size_t widened_kv_bytes(const attn_args* a) {
+  return align256((size_t)a->n_cells * a->n_head_kv * a->head_dim * 2);
+}
+size_t widened_q_bytes(const attn_args* a) {
+  return a->q_type == ATTN_BF16 ? align256((size_t)a->n_rows * a->n_head_q * a->head_dim * 2) : 0;
+}
+size_t widened_bytes(const attn_args* a) { return 2 * widened_kv_bytes(a) + widened_q_bytes(a); }
+attn_args widened_args(const attn_args* a, void* ws) {
+  attn_args b = *a;
+  char* base = static_cast<char*>(ws);
+  b.k = base;
+  b.v = base ? base + widened_kv_bytes(a) : nullptr;
+  b.kv_type = ATTN_F16;
+  b.kv_stride_cell = (int64_t)a->n_head_kv * a->head_dim;
+  b.kv_stride_head = a->head_dim;
+  b.k_scale = b.v_scale = nullptr;
+  b.scale_stride_cell = 0;
+  if (a->q_type == ATTN_BF16) {
+    b.q = base ? base + 2 * widened_kv_bytes(a) : reinterpret_cast<void*>(static_cast<uintptr_t>(256));
+    b.q_type = ATTN_F16;
+    b.q_stride_row = (int64_t)a->n_head_q * a->head_dim;
+    b.q_stride_head = a->head_dim;
+  }
+  return b;
+}
+
 int32_t attn_supports(const attn_args* a, int32_t op) {
   switch (op) {
     case ATTN_OP_DECODE: return check_decode(a);
@@ -614,8 +654,12 @@ size_t attn_workspace_size(const attn_args* a, int32_t op, int32_t n_sel) {
     case ATTN_OP_SELECTED:
       if (n_sel < 1 || n_sel > kMaxSel) return 0;
       return selected_ws_layout(a, n_sel, plan_selected(a, n_sel, sms)).total;
-    case ATTN_OP_PREFILL:
-      return unified_route(a) ? unified_ws_bytes(a, sms) : prefill_ws_layout(a, plan_prefill_split(a, sms)).total;
+    case ATTN_OP_PREFILL: {
+      if (unified_route(a)) return unified_ws_bytes(a, sms);
+      if (!is_quantized(a->kv_type)) return prefill_ws_layout(a, plan_prefill_split(a, sms)).total;
+      const attn_args b = widened_args(a, nullptr);
+      return widened_bytes(a) + prefill_ws_layout(&b, plan_prefill_split(&b, sms)).total;
+    }
     case ATTN_OP_SELECTED_MASKED: {
       if (n_sel < 1 || n_sel > kMaxSel) return 0;
       const attn_args pa = sel_mask_args(a, reinterpret_cast<float*>(static_cast<uintptr_t>(256)));
@@ -902,6 +946,9 @@ int32_t attn_prefill(const attn_args* a, void* ws, size_t ws_bytes, void* stream
   return attn_prefill_timed(a, ws, ws_bytes, stream, nullptr);
 }
 
+int32_t prefill_dense(const attn_args* a, void* ws, size_t ws_bytes, void* stream, void* const events[3],
+                      DeviceInfo* di, bool started);
+
 int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* stream, void* const events[3]) {
   int32_t st = check_prefill(a);
   if (st != ATTN_OK) return st;
@@ -909,6 +956,41 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != ATTN_OK) return st;
   if (unified_route(a)) return run_unified(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), events, di);
+  if (!is_quantized(a->kv_type)) return prefill_dense(a, ws, ws_bytes, stream, events, di, false);
+  // e4m3 / int8 cache: widen K and V into the workspace, then the dense path
+  // (sequence ids included: its classifier applies them)
+  const size_t wb = widened_bytes(a);
+  if (ws == nullptr || ws_bytes < wb)
+    return fail(ATTN_ERR_WORKSPACE, "prefill over an e4m3/int8 cache needs %zu workspace bytes for the widened "
+                "K/V, got %zu", wb, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(ATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const attn_args b = widened_args(a, ws);
+  {   // the rest of the workspace must hold the dense path's part before anything is launched
+    const PrefillWs wl = prefill_ws_layout(&b, plan_prefill_split(&b, di->sms));
+    if (ws_bytes - wb < wl.total)
+      return fail(ATTN_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", wb + wl.total, ws_bytes);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  record_event(events, 0, s);
+  DequantPlan dp{};
+  dp.N = a->n_cells; dp.Hkv = a->n_head_kv; dp.D = a->head_dim;
+  dp.code_type = a->kv_type;
+  dp.k = a->k; dp.v = a->v; dp.sc = a->kv_stride_cell; dp.sh = a->kv_stride_head;
+  dp.k_scale = a->k_scale; dp.v_scale = a->v_scale; dp.ss = a->scale_stride_cell;
+  dp.k_out = const_cast<void*>(b.k); dp.v_out = const_cast<void*>(b.v);
+  dp.R = a->n_rows; dp.Hq = a->n_head_q;
+  dp.q = a->q; dp.q_sr = a->q_stride_row; dp.q_sh = a->q_stride_head;
+  dp.q_out = a->q_type == ATTN_BF16 ? const_cast<void*>(b.q) : nullptr;
+  cudaError_t e = launch_dequant(dp, di->sms, s);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "widening launch: %s", cudaGetErrorString(e));
+  return prefill_dense(&b, static_cast<char*>(ws) + wb, ws_bytes - wb, stream, events, di, true);
+}
+
+// The tensor-core path over a 16-bit cache (started: event 0 was recorded by
+// the caller, ahead of its own kernels).
+int32_t prefill_dense(const attn_args* a, void* ws, size_t ws_bytes, void* stream, void* const events[3],
+                      DeviceInfo* di, bool started) {
+  int32_t st = ATTN_OK;
   const PrefillSplit sp = plan_prefill_split(a, di->sms);
   const PrefillWs wl = prefill_ws_layout(a, sp);
   if (wl.total > 0 && (ws == nullptr || ws_bytes < wl.total))
@@ -1017,7 +1099,7 @@ int32_t attn_prefill_timed(const attn_args* a, void* ws, size_t ws_bytes, void* 
   p.test_stall = a->reserved[0] > 0 ? 1 : 0;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  record_event(events, 0, s);
+  if (!started) record_event(events, 0, s);
   cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, s, nullptr);
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
   record_event(events, 1, s);

@@ -200,6 +200,23 @@ struct PrefillPlan {
   int32_t test_stall;       // 1: the softmax warps first wait on a barrier nothing arrives at
 };
 
+// ---- widening of e4m3 / int8 caches for prefill ------------------------------
+struct DequantPlan {
+  int32_t N, Hkv, D;
+  int32_t code_type;        // ATTN_FP8_E4M3 or ATTN_I8 (widened to F16)
+  const void *k, *v;        // codes [N][Hkv][D] with strides sc, sh (bytes = elements)
+  int64_t sc, sh;
+  const float *k_scale, *v_scale;   // [N][ss], column = KV head
+  int64_t ss;
+  void *k_out, *v_out;      // [N][Hkv][D] contiguous, F16
+  // a BF16 Q copied to F16 ([R][Hq][D] contiguous), or q_out NULL
+  int32_t R, Hq;
+  const void* q;
+  int64_t q_sr, q_sh;
+  void* q_out;
+};
+cudaError_t launch_dequant(const DequantPlan& p, int sms, cudaStream_t stream);
+
 cudaError_t launch_prefill(const PrefillPlan& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, cudaStream_t stream, cudaEvent_t after_classify);
 

@@ -36,6 +36,7 @@ the path has no collective); only a scalar max of the step time crosses ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -530,6 +531,34 @@ def run_parts(args, rank, dev, stream, with_cpu=False):
         parts["prefill"]["cpu_baseline"] = _part_baseline(p, [128 * i + 64 for i in range(16)], prefill_flops,
                                                           "TFLOP/s", 1e12, "16 of the 2048 rows (one per row tile)")
     del q, k, v, out, pa, ws, kw
+
+    # the causal prefill workload over an e4m3 cache (K and V quantized per
+    # (cell, KV head), amax / 448): attn_prefill widens the codes into its
+    # workspace and runs the same tensor-core path; TensorFold PR #911 puts
+    # its e4m3 prefill within 5% of bf16.
+    pq = W.causal_prefill()
+    kq, ksq = W.quantize_kv(pq.k.to(torch.float32), "e4m3")
+    vq, vsq = W.quantize_kv(pq.v.to(torch.float32), "e4m3")
+    pq = dataclasses.replace(pq, k=kq, v=vq, k_scale=ksq, v_scale=vsq)
+    (q, k, v, out), kw = A.problem_kwargs(pq, device=dev)
+    pa = A.make_args(q, k, v, out, **kw)
+    ws = torch.empty(max(A.workspace_size(pa, A.OP_PREFILL), 256), dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        A.attn_prefill_args(pa, ws=ws, stream=stream)
+    whole_q, main_q = _time_calls(lambda e: A.attn_prefill_timed_args(pa, ws, e, stream=stream), n, flush, stream)
+    parts["fp8_prefill"] = {
+        "workload": "causal_prefill over an e4m3 cache (per (cell, KV head) F32 scales): widening kernel + the "
+                    "bf16 tensor-core prefill",
+        "value": flops / (whole_q * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_per_call": whole_q, "vs_bf16_prefill": whole_q / parts["prefill"]["ms_per_call"], "calls": n,
+        "gpu_launches": 3 * n,   # widening + classifier + tensor-core kernel
+        "roofline": {"bound": "tensor", "achieved": flops / (main_q * 1e-3) / 1e12, "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": flops / (main_q * 1e-3) / 1e12 / tc_peak, "traffic": None,
+                     "kernel": "dequant_kernel + prefill_classify_kernel + prefill_kernel (tcgen05)",
+                     "kernel_ms": main_q, "algorithmic_flops": flops,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst cuBLAS)"},
+    }
+    del q, k, v, out, pa, ws, kw, pq, kq, vq
 
     # draft-tree decode rows: 16 nodes of a binary draft tree over 130856 keys
     # (the depth of TensorFold PR #2595's long-context receipt), GQA heads;

@@ -98,7 +98,7 @@
  * K and V base addresses and their cell/head strides must be 16-byte
  * aligned (tile loads by the Tensor Memory Accelerator).
  *
- * Quantized caches (attn_decode only; TensorFold PR #911: e4m3 rows with one
+ * Quantized caches (attn_decode and attn_prefill; TensorFold PR #911: e4m3 rows with one
  * fp32 scale per (position, key head) = amax / 448, half the bytes of bf16;
  * TensorFold PR #2595: an int8 cache with a K scale and a V scale per key).
  * With kv_type ATTN_FP8_E4M3 or ATTN_I8 the stored codes are one byte each and
@@ -113,7 +113,16 @@
  * 8 elements), head_dim 128 or 256 and at most 8 query heads per KV head, the
  * codes run on the tensor cores (widened to f16 in registers, which is exact);
  * other shapes and forced slice counts run on the CUDA cores.
- * attn_selected and attn_prefill refuse quantized caches (ATTN_ERR_UNSUPPORTED).
+ * attn_prefill takes them with Q in F16 or BF16: one
+ * kernel writes code x scale, rounded once to F16, into a contiguous
+ * [n_cells][n_head_kv][head_dim] copy of K and of V at the start of the
+ * workspace (as TensorFold PR #911's prefill stages e4m3 rows widened to
+ * bf16; F16 keeps the one rounding well inside the tolerances), a BF16 Q is
+ * copied to F16 after them (the tensor cores take both operands in one type),
+ * and the F16 tensor-core prefill runs on the copies.  Values beyond F16's
+ * range (|x| > 65504) become infinite.  K, V and their strides must be
+ * 16-byte aligned.  attn_selected refuses quantized caches
+ * (ATTN_ERR_UNSUPPORTED).
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H

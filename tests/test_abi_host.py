@@ -132,13 +132,27 @@ def test_bounded_wait_test_field(lib):
 
 
 def test_quantized_cache_validation(lib):
-    """e4m3/int8 caches: decode only, scales required, and only for such caches."""
+    """e4m3/int8 caches: decode and prefill (with a 16-bit Q and 16-byte
+    aligned codes), scales required, and only for such caches; the prefill
+    workspace holds the K and V widened to the Q dtype."""
     for kv in (A.ATTN_FP8_E4M3, A.ATTN_I8):
         a = _args(kv_type=kv, kv_stride_cell=2 * 128, kv_stride_head=128)
         assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1      # scales missing
         a.k_scale, a.v_scale, a.scale_stride_cell = 0x60000, 0x70000, a.n_head_kv
         assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == 0
-        assert lib.attn_supports(ctypes.byref(a), A.OP_PREFILL) == -2
+        assert lib.attn_supports(ctypes.byref(a), A.OP_PREFILL) == 0
+        widened = 2 * a.n_cells * a.n_head_kv * a.head_dim * 2
+        assert lib.attn_workspace_size(ctypes.byref(a), A.OP_PREFILL, 0) >= widened
+        assert lib.attn_supports(ctypes.byref(a), A.OP_SELECTED) == -2
+        b = _args(kv_type=kv, kv_stride_cell=2 * 128, kv_stride_head=128, k_scale=0x60000, v_scale=0x70000,
+                  scale_stride_cell=2, q_type=A.ATTN_F32)
+        assert lib.attn_supports(ctypes.byref(b), A.OP_PREFILL) == -2     # Q must be F16/BF16 here
+        b = _args(kv_type=kv, kv_stride_cell=2 * 128 + 8, kv_stride_head=128, k_scale=0x60000, v_scale=0x70000,
+                  scale_stride_cell=2)
+        assert lib.attn_supports(ctypes.byref(b), A.OP_PREFILL) == -2     # codes not 16-byte aligned
+        b = _args(kv_type=kv, kv_stride_cell=2 * 128, kv_stride_head=128, k_scale=0x60000, v_scale=0x70000,
+                  scale_stride_cell=2, cell_seq=0x50000, row_seq=0x58000)
+        assert lib.attn_supports(ctypes.byref(b), A.OP_PREFILL) == 0      # sequence ids: the dense path's filter
         a.scale_stride_cell = a.n_head_kv - 1
         assert lib.attn_supports(ctypes.byref(a), A.OP_DECODE) == -1
     a = _args()
