@@ -113,34 +113,41 @@ __device__ __forceinline__ void pf_classify_tile(const PrefillPlan& p, int64_t b
       cs[e] = (cin[e] && p.f.cell_seq) ? __ldg(p.f.cell_seq + c) : 0;
       cpg[e] = (cin[e] && p.f.cell_pos) ? __ldg(p.f.cell_pos + c) : 0;
     }
-    float4 mv[kClsRowsPerWarp];
+    // the 16 rows of each warp in two batches of 8: a batch's 16-byte mask
+    // loads all go out before any is used, and the smaller register set lets
+    // four CTAs share an SM
+    bool any = false, notfull = false, bias = false, late = false;
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+    float4 mv[kClsRowsPerWarp / 2];
     if (p.f.mask) {
       const bool vec = p.mask_vec && kt * kPfCells + kPfCells <= p.N;
 #pragma unroll
-      for (int i = 0; i < kClsRowsPerWarp; ++i) {
+      for (int i2 = 0; i2 < kClsRowsPerWarp / 2; ++i2) {
+        const int i = hb * (kClsRowsPerWarp / 2) + i2;
         const int r = rt * p.rpt + warp + 8 * i;
-        mv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        mv[i2] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (warp + 8 * i < p.rpt && r < p.R) {
           const float* mrow = p.f.mask + (int64_t)r * p.f.mask_sr + c_base;
           if (vec) {
-            mv[i] = __ldg(reinterpret_cast<const float4*>(mrow));
+            mv[i2] = __ldg(reinterpret_cast<const float4*>(mrow));
           } else {
-            if (cin[0]) mv[i].x = __ldg(mrow);
-            if (cin[1]) mv[i].y = __ldg(mrow + 1);
-            if (cin[2]) mv[i].z = __ldg(mrow + 2);
-            if (cin[3]) mv[i].w = __ldg(mrow + 3);
+            if (cin[0]) mv[i2].x = __ldg(mrow);
+            if (cin[1]) mv[i2].y = __ldg(mrow + 1);
+            if (cin[2]) mv[i2].z = __ldg(mrow + 2);
+            if (cin[3]) mv[i2].w = __ldg(mrow + 3);
           }
         }
       }
     }
-    __syncthreads();
-    bool any = false, notfull = false, bias = false, late = false;
+    if (hb == 0) __syncthreads();   // the rows' data staged
 #pragma unroll
-    for (int i = 0; i < kClsRowsPerWarp; ++i) {
+    for (int i2 = 0; i2 < kClsRowsPerWarp / 2; ++i2) {
+      const int i = hb * (kClsRowsPerWarp / 2) + i2;
       const int rl = warp + 8 * i;
       if (rl >= p.rpt || rt * p.rpt + rl >= p.R) continue;   // warp-uniform
       const int4 rv = rows_sh[rl];
-      const float mvals[4] = {mv[i].x, mv[i].y, mv[i].z, mv[i].w};
+      const float mvals[4] = {mv[i2].x, mv[i2].y, mv[i2].z, mv[i2].w};
       uint32_t nib = 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -168,6 +175,7 @@ __device__ __forceinline__ void pf_classify_tile(const PrefillPlan& p, int64_t b
         if ((lane & 7) == 0) p.bits[((b * kPfRows + rl) << 2) + (lane >> 3)] = word;
       }
     }
+    }
     const int a = __syncthreads_or(any ? 1 : 0);
     const int nf = __syncthreads_or(notfull ? 1 : 0);
     const int bs = __syncthreads_or(bias ? 1 : 0);
@@ -187,7 +195,7 @@ __device__ __forceinline__ void pf_scan_tile(const PrefillPlan& p, int kt, int g
     // per_row consecutive lanes; per_row divides 32).
     const int per_row = p.D / 8;
     const int n_chunk = kPfCells * per_row;
-    constexpr int kPer = 8;   // chunks per thread per round (all loads of a round go out first)
+    constexpr int kPer = 4;   // chunks per thread per round (all loads of a round go out first)
     const uint16_t* vbase = static_cast<const uint16_t*>(p.v) + (int64_t)g * p.kv_sh;
     const uint16_t* kbase = static_cast<const uint16_t*>(p.k) + (int64_t)g * p.kv_sh;
     // A 16-bit value is non-finite iff its exponent field is all ones.
@@ -254,7 +262,7 @@ __device__ __forceinline__ void pf_scan_tile(const PrefillPlan& p, int kt, int g
 
 // Blocks b < n_rt * n_kt classify tile b; the blocks after them scan one
 // (cell tile, KV head) each.
-__global__ void __launch_bounds__(kClsThreads) prefill_classify_kernel(PrefillPlan p) {
+__global__ void __launch_bounds__(kClsThreads, 4) prefill_classify_kernel(PrefillPlan p) {
   pdl_launch_dependents();   // the prefill kernel may start its prologue
   __shared__ int4 rows_sh[kPfRows];
   __shared__ float wmax[kClsThreads / 32];
