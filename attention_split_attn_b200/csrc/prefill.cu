@@ -928,7 +928,14 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
   bool ok = true;
   float qn2 = 0.f;   // |q_r|^2 of this row and head (softcap range bound)
   for (int kt = tiles.first(); kt >= 0; kt = tiles.next(kt), ++j) {
+    // the tile's class, K-tile norm and this row's visibility bits are read
+    // before the wait for S, so their latency overlaps it
     const int code = tiles.code(kt);
+    const bool bits_tile = tiles.bits(kt);
+    const float kn2_t = p.kn2 ? __ldg(p.kn2 + (int64_t)kt * p.Hkv + tiles.g) : 0.f;
+    const uint4 bw = (bits_tile && rvalid) ? __ldg(reinterpret_cast<const uint4*>(
+                                                 p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_l) << 2)))
+                                           : make_uint4(0u, 0u, 0u, 0u);
     if (!pf_wait_warp(&s_full[slot], (uint32_t)(j & 1), p, abort_flag)) { ok = false; break; }
     tc_fence_after();
     if (j == 0 && p.kn2) {
@@ -960,7 +967,6 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
     // positions and no visible cell after its row (see pf_transform_fast).
     // Each path below reads S, computes the logits and then the weights on
     // its own, so only P crosses the join (it keeps register use low).
-    const bool bits_tile = tiles.bits(kt);
     bool fast = (code == kTileFull || bits_tile) && (!cap || p.cap_raw) &&
                 (al == 0 || (al == 1 && !tiles.late(kt)));
     bool done = false;
@@ -973,7 +979,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
         // The softcap series of degree 7 where |u| <= c / 3 for every row of
         // the warp (truncation below 1e-6 c), degree 9 where |u| <= 0.4 c
         // (below 3.7e-7 c).
-        const float qk2 = qn2 * __ldg(p.kn2 + (int64_t)kt * p.Hkv + tiles.g);
+        const float qk2 = qn2 * kn2_t;
         int deg = -1;
         if (cap) deg = __all_sync(0xffffffffu, qk2 <= p.bound7) ? 7 : __all_sync(0xffffffffu, qk2 <= p.bound9) ? 9 : -1;
         else deg = __all_sync(0xffffffffu, qk2 <= p.nc_lim2) ? 0 : -1;
@@ -984,9 +990,6 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
           // visible cells of this row in the tile: all (full) or the stored bits
           int i_lo = 0, i_hi = kPfCells - 1;
           if (bits_tile) {
-            const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
-                                          p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_l) << 2)))
-                                    : make_uint4(0u, 0u, 0u, 0u);
             vis[0] = bw.x; vis[1] = bw.y; vis[2] = bw.z; vis[3] = bw.w;
             i_hi = vis[3] ? 96 + 31 - __clz(vis[3]) : vis[2] ? 64 + 31 - __clz(vis[2])
                  : vis[1] ? 32 + 31 - __clz(vis[1]) : vis[0] ? 31 - __clz(vis[0]) : -1;
@@ -1041,7 +1044,7 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       float x[kPfCells], mt, smax = 0.f;
       // every row's |q|^2 max |k|^2 within range: no per-cell check
       const bool bounded = cap && p.kn2 != nullptr &&
-                           __all_sync(0xffffffffu, qn2 * __ldg(p.kn2 + (int64_t)kt * p.Hkv + tiles.g) <= p.bound2);
+                           __all_sync(0xffffffffu, qn2 * kn2_t <= p.bound2);
       if (bounded) {
         if (al == 1) pf_transform_fast<2, true>(raw, x, p, slope, C, mt, smax);
         else pf_transform_fast<2, false>(raw, x, p, slope, C, mt, smax);
@@ -1059,9 +1062,6 @@ __device__ __forceinline__ void pf_softmax(const PrefillPlan& p, const PfTiles& 
       } else {
         const float boff = al == 1 ? C : 0.f, bstep = al == 1 ? 8.f * slope : 0.f;
         if (bits_tile) {
-          const uint4 bw = rvalid ? __ldg(reinterpret_cast<const uint4*>(
-                                        p.bits + ((((int64_t)rt * p.n_kt + kt) * kPfRows + row_l) << 2)))
-                                  : make_uint4(0u, 0u, 0u, 0u);
           vis[0] = bw.x; vis[1] = bw.y; vis[2] = bw.z; vis[3] = bw.w;
           pf_apply_bits(x, vis, boff, bstep, mt);
         }
